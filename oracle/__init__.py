@@ -1,0 +1,115 @@
+"""fp64 CPU oracle for the fused attention forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline / reference leg of
+``bench.py`` may import this package.  The product path (the CUDA library and its
+Python binding) never imports, links or calls it, and shares no code with it.
+
+The arithmetic lives in ``attn_ref.c`` (plain C, fp64, libm ``exp``/``log``, no
+fast-math); this module only marshals numpy arrays through ctypes.  It follows the
+softmax-attention definition that the TileLang tutorial's FlashAttention section
+validates against (pro.edgex.exchange summary, FlashAttention paragraph; datastack.it,
+"Cosa copre il tutorial": causal and non-causal):
+
+    O = softmax(scale * Q K^T  [+ top-left causal mask]) V
+    LSE_i = ln sum_j exp(scale * q_i . k_j)     (over the unmasked j)
+
+Pins (see tests/test_oracle_pins.py): closed forms (Sk = 1, Q = 0, constant V,
+causal row 0, one-hot attention), invariants (row sums, permutation and shift
+invariance), hand-derived tiny cases, and PyTorch's float64 math SDPA on the CPU.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+ORACLE_OK = 0
+ORACLE_ERR_ARGS = 1
+ORACLE_ERR_NOMEM = 2
+ORACLE_ERR_ROWSUM = 3
+
+_LIB = None
+
+
+def _bind(path):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lp = ctypes.c_long
+    lib.attn_ref_f64.argtypes = [dp, dp, dp, dp, dp, dp, lp, lp, lp, lp, lp,
+                                 ctypes.c_int, ctypes.c_double]
+    lib.attn_ref_f64.restype = ctypes.c_int
+    lib.attn_ref_rows_f64.argtypes = [dp, dp, dp, ctypes.POINTER(ctypes.c_int64), lp,
+                                      dp, dp, lp, lp, lp, lp, lp, ctypes.c_int,
+                                      ctypes.c_double]
+    lib.attn_ref_rows_f64.restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def load(path=None):
+    """Load (building first if needed) the oracle library, or the one at `path`."""
+    global _LIB
+    if path is not None:
+        return _bind(path)
+    if _LIB is None:
+        _LIB = _bind(_build.build())
+    return _LIB
+
+
+def _f64(a):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads(lib=None):
+    return (lib or load()).oracle_num_threads()
+
+
+def attn_ref(q, k, v, causal, scale, return_probs=False, lib=None):
+    """Whole problem.  q: [B,H,Sq,D], k, v: [B,H,Sk,D] (any real dtype, upcast
+    exactly to fp64).  Returns (O [B,H,Sq,D], LSE [B,H,Sq]) in fp64, plus the
+    probability matrices [B,H,Sq,Sk] when return_probs."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    if k.shape != (B, H, Sk, D) or v.shape != (B, H, Sk, D):
+        raise ValueError("k and v must be [B,H,Sk,D] with q's B, H, D")
+    o = np.empty((B, H, Sq, D), dtype=np.float64)
+    lse = np.empty((B, H, Sq), dtype=np.float64)
+    p = np.empty((B, H, Sq, Sk), dtype=np.float64) if return_probs else None
+    rc = lib.attn_ref_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                          _ptr(p) if p is not None else None,
+                          B, H, Sq, Sk, D, int(bool(causal)), float(scale))
+    if rc != ORACLE_OK:
+        raise RuntimeError(f"oracle attn_ref_f64 failed with code {rc}")
+    return (o, lse, p) if return_probs else (o, lse)
+
+
+def attn_ref_rows(q, k, v, rows, causal, scale, lib=None):
+    """Selected query rows only.  rows: int array [n, 3] of (b, h, i).
+    Returns (O [n, D], LSE [n]) in fp64."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = lib.attn_ref_rows_f64(_ptr(q), _ptr(k), _ptr(v),
+                               rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n,
+                               _ptr(o), _ptr(lse), B, H, Sq, Sk, D,
+                               int(bool(causal)), float(scale))
+    if rc != ORACLE_OK:
+        raise RuntimeError(f"oracle attn_ref_rows_f64 failed with code {rc}")
+    return o, lse
+
+
+__all__ = ["attn_ref", "attn_ref_rows", "load", "num_threads"]
