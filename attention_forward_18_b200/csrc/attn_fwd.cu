@@ -1,0 +1,268 @@
+// attn_fwd.cu -- host side of the C ABI declared in include/attn_fwd.h: argument
+// checks, TMA descriptor encoding, kernel selection and launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn_fwd.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxSeq = 1 << 24;
+constexpr int kMaxHeads = 1 << 24;
+constexpr int kMaxDevices = 64;
+
+// cuTensorMapEncodeTiled, fetched through the runtime so the library needs no
+// link against libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [BH, S, D] 16-bit tensor seen as 3-D (D innermost); box = 64 elements (128 bytes,
+// the swizzle span) x 128 rows x 1 head; rows past S read as zeros.
+bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(S) * D * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(attn::CHUNK_ELEMS),
+                               static_cast<cuuint32_t>(attn::BN), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r =
+        fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Per-device facts checked once: compute capability 10.x.
+int check_device() {
+    static int verdict[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return ATTN_ERR_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (verdict[dev] == 0) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return ATTN_ERR_DEVICE;
+        }
+        verdict[dev] = (major == 10) ? 1 : -1;
+    }
+    return verdict[dev] == 1 ? ATTN_OK : ATTN_ERR_DEVICE;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             int B, int H, int Sq, int Sk, int D, float scale, int dtype) {
+    if (!q || !k || !v || !o) return ATTN_ERR_NULLPTR;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
+    if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
+    if (B < 1 || H < 1 || Sq < 1 || Sk < 1) return ATTN_ERR_SHAPE;
+    if (Sq > kMaxSeq || Sk > kMaxSeq) return ATTN_ERR_SHAPE;
+    const int64_t bh = static_cast<int64_t>(B) * H;
+    if (bh > kMaxHeads) return ATTN_ERR_SHAPE;
+    const int64_t n_qb = (Sq + attn::BM - 1) / attn::BM;
+    if (n_qb * bh > INT_MAX) return ATTN_ERR_SHAPE;
+    if (!std::isfinite(scale)) return ATTN_ERR_SCALE;
+    auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+    if (mis16(q) || mis16(k) || mis16(v) || mis16(o)) return ATTN_ERR_ALIGN;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_ALIGN;
+    const size_t nq = static_cast<size_t>(bh) * Sq * D * 2;
+    const size_t nk = static_cast<size_t>(bh) * Sk * D * 2;
+    if (overlaps(o, nq, q, nq) || overlaps(o, nq, k, nk) || overlaps(o, nq, v, nk))
+        return ATTN_ERR_ALIAS;
+    if (lse) {
+        const size_t nl = static_cast<size_t>(bh) * Sq * 4;
+        if (overlaps(lse, nl, q, nq) || overlaps(lse, nl, k, nk) || overlaps(lse, nl, v, nk) ||
+            overlaps(lse, nl, o, nq))
+            return ATTN_ERR_ALIAS;
+    }
+    return ATTN_OK;
+}
+
+template <int D, int NS, bool BF16, bool CAUSAL>
+int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const attn::Params& p, int grid, cudaStream_t stream) {
+    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL>;
+    constexpr int smem = attn::SmemLayout<D, NS>::ALLOC;
+    static bool attr_set[kMaxDevices];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_LAUNCH;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            attr_set[dev] = true;
+        }
+    }
+    kern<<<grid, attn::NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// Ring depth: as many K/V stages as fit beside the Q tile while keeping the
+// shared-memory request above half an SM (one CTA per SM).
+template <int D>
+constexpr int kStages = (D == 64) ? 4 : 2;
+
+template <int D, bool BF16>
+int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+             const attn::Params& p, int grid, bool causal, cudaStream_t s) {
+    if (causal) return launch_one<D, kStages<D>, BF16, true>(tq, tk, tv, p, grid, s);
+    return launch_one<D, kStages<D>, BF16, false>(tq, tk, tv, p, grid, s);
+}
+
+int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+        int Sk, int D, int causal, float scale, int dtype, cudaStream_t stream, unsigned flags) {
+    int rc = validate(q, k, v, o, lse, B, H, Sq, Sk, D, scale, dtype);
+    if (rc != ATTN_OK) return rc;
+    if ((rc = check_device()) != ATTN_OK) return rc;
+
+    const int BH = B * H;
+    const bool bf16 = dtype == ATTN_BF16;
+    CUtensorMap tq, tk, tv;
+    if (!encode_qkv_map(&tq, q, D, Sq, BH, bf16) || !encode_qkv_map(&tk, k, D, Sk, BH, bf16) ||
+        !encode_qkv_map(&tv, v, D, Sk, BH, bf16))
+        return ATTN_ERR_TENSORMAP;
+
+    attn::Params p;
+    p.o = o;
+    p.lse = lse;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.BH = BH;
+    p.n_qb = (Sq + attn::BM - 1) / attn::BM;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+    p.flags = flags;
+    const int grid = p.n_qb * BH;
+    const bool c = causal != 0;
+    if (D == 64) return bf16 ? launch_d<64, true>(tq, tk, tv, p, grid, c, stream)
+                             : launch_d<64, false>(tq, tk, tv, p, grid, c, stream);
+    return bf16 ? launch_d<128, true>(tq, tk, tv, p, grid, c, stream)
+                : launch_d<128, false>(tq, tk, tv, p, grid, c, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int Sq, int Sk, int D, int causal, float scale, int dtype, attn_stream_t stream) {
+    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+               reinterpret_cast<cudaStream_t>(stream), 0u);
+}
+
+int attn_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int H, int Sq, int Sk, int D, int causal, float scale, int dtype,
+                   attn_stream_t stream, unsigned flags) {
+    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+               reinterpret_cast<cudaStream_t>(stream), flags & attn::FLAG_SKIP_Q_LOAD);
+}
+
+int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                  float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                  float* lse_dev, int B, int H, int Sq, int Sk, int D, int causal, float scale,
+                  int dtype, attn_stream_t stream) {
+    if (!q_host || !k_host || !v_host || !o_host) return ATTN_ERR_NULLPTR;
+    int rc = validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Sq, Sk, D, scale, dtype);
+    if (rc != ATTN_OK) return rc;
+    if ((rc = check_device()) != ATTN_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t bh = static_cast<size_t>(B) * H;
+    const size_t nq = bh * Sq * D * 2, nk = bh * Sk * D * 2;
+    if (cudaMemcpyAsync(q_dev, q_host, nq, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(k_dev, k_host, nk, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(v_dev, v_host, nk, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    rc = run(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Sq, Sk, D, causal, scale, dtype, s, 0u);
+    if (rc != ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o_host, o_dev, nq, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    if (lse_host && lse_dev &&
+        cudaMemcpyAsync(lse_host, lse_dev, bh * Sq * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    return ATTN_OK;
+}
+
+int attn_fwd_status(attn_stream_t stream, int* device_status) {
+    if (!device_status) return ATTN_ERR_NULLPTR;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int value = 0;
+    const int zero = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&value, attn::g_attn_status, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(attn::g_attn_status, &zero, sizeof(int), 0,
+                                cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    *device_status = value;
+    return ATTN_OK;
+}
+
+const char* attn_fwd_strerror(int code) {
+    switch (code) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_NULLPTR: return "null pointer argument";
+        case ATTN_ERR_ALIGN: return "misaligned pointer (q/k/v/o need 16 bytes, lse 4)";
+        case ATTN_ERR_SHAPE: return "bad shape (B, H, Sq, Sk >= 1 and within limits)";
+        case ATTN_ERR_HEADDIM: return "unsupported head dimension (64 or 128)";
+        case ATTN_ERR_DTYPE: return "unsupported dtype (ATTN_F16 or ATTN_BF16)";
+        case ATTN_ERR_TENSORMAP: return "TMA descriptor encoding failed";
+        case ATTN_ERR_LAUNCH: return "CUDA call or kernel launch failed";
+        case ATTN_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+        case ATTN_ERR_SCALE: return "scale is not finite";
+        case ATTN_ERR_ALIAS: return "output overlaps an input";
+        case ATTN_ERR_DEVICE: return "no usable sm_100 CUDA device";
+        default: return "unknown error code";
+    }
+}
+
+int attn_fwd_abi_version(void) { return 1; }
+
+}  // extern "C"

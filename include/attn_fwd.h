@@ -1,0 +1,117 @@
+/*
+ * attn_fwd.h -- C ABI of the B200 (sm_100a) fused attention forward pass.
+ *
+ * The operation ("Designing High-Performance GPU Kernels with TileLang"; the
+ * FlashAttention paragraph of the pro.edgex.exchange summary and "Cosa copre il
+ * tutorial" on datastack.it): for every batch b, head h and query row i,
+ *
+ *     s_ij   = scale * sum_d Q[b,h,i,d] K[b,h,j,d]
+ *     s_ij   = -inf  when causal and j > i          (top-left aligned mask)
+ *     O[b,h,i,:] = sum_j softmax_j(s_i.) V[b,h,j,:]
+ *     LSE[b,h,i] = ln sum_j exp(s_ij)                (natural log, scaled scores)
+ *
+ * computed tile by tile with an online softmax so the Sq x Sk score matrix never
+ * reaches device memory.  The pages fix neither the layout, the mask alignment
+ * for Sq != Sk, nor the log-sum-exp output; the choices below are this library's.
+ *
+ * Layout: Q [B,H,Sq,D], K and V [B,H,Sk,D], O [B,H,Sq,D], all contiguous
+ * row-major 16-bit (one dtype for all four); LSE [B,H,Sq] contiguous fp32.
+ * Arithmetic: 16-bit operands, fp32 accumulation and softmax, one rounding of O.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates no memory and
+ * keeps no pointer after a call returns.  Device-pointer calls are asynchronous on
+ * `stream` (the stream's previous work completes first; nothing else is
+ * synchronised).
+ *
+ * Errors: argument errors return a negative code before any CUDA call and leave
+ * every buffer untouched.  A failed launch returns ATTN_ERR_LAUNCH.  A kernel whose
+ * pipeline wait runs out of time (2 s per wait) stops, records ATTN_ERR_TIMEOUT in
+ * the per-device status word (read it with attn_fwd_status) and leaves O / LSE
+ * undefined; nothing traps or aborts.
+ */
+#ifndef ATTN_FWD_H
+#define ATTN_FWD_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; a null stream is the legacy default stream. */
+typedef struct CUstream_st *attn_stream_t;
+
+/* Element type of Q, K, V and O. */
+typedef enum { ATTN_F16 = 0, ATTN_BF16 = 1 } attn_dtype_t;
+
+enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULLPTR = -1,   /* q, k, v or o is null                                */
+    ATTN_ERR_ALIGN = -2,     /* q, k, v, o not 16-byte aligned, or lse not 4-byte   */
+    ATTN_ERR_SHAPE = -3,     /* B, H, Sq or Sk < 1, or a size beyond the limits     */
+    ATTN_ERR_HEADDIM = -4,   /* D is not 64 or 128                                  */
+    ATTN_ERR_DTYPE = -5,     /* dtype is not ATTN_F16 / ATTN_BF16                   */
+    ATTN_ERR_TENSORMAP = -6, /* the driver refused a TMA descriptor                 */
+    ATTN_ERR_LAUNCH = -7,    /* a CUDA call or the kernel launch failed             */
+    ATTN_ERR_TIMEOUT = -8,   /* (status word) a pipeline wait ran out of time       */
+    ATTN_ERR_SCALE = -9,     /* scale is NaN or infinite                            */
+    ATTN_ERR_ALIAS = -10,    /* o or lse overlaps q, k or v                         */
+    ATTN_ERR_DEVICE = -11    /* no CUDA device, or the current one is not sm_100    */
+};
+
+/*
+ * attn_fwd -- O and LSE from device buffers.
+ *   q      device, [B,H,Sq,D] 16-bit, 16-byte aligned
+ *   k, v   device, [B,H,Sk,D] 16-bit, 16-byte aligned
+ *   o      device, [B,H,Sq,D] 16-bit, 16-byte aligned, written; must not overlap q/k/v
+ *   lse    device, [B,H,Sq] fp32, written; may be NULL (not written)
+ *   B, H, Sq, Sk >= 1; B*H, Sq, Sk <= 2^24; D in {64, 128}
+ *   causal 0: every key visible; nonzero: key j visible to query i iff j <= i
+ *   scale  finite multiplier of q.k (e.g. 1/sqrt(D)); |scale*q.k| must fit fp32
+ *   dtype  ATTN_F16 or ATTN_BF16
+ *   stream the CUDA stream to run on
+ * Returns ATTN_OK once the kernel is queued, or a negative code (see above).
+ */
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+             int B, int H, int Sq, int Sk, int D, int causal, float scale,
+             int dtype, attn_stream_t stream);
+
+/*
+ * attn_fwd_host -- the same pass from host buffers: copies q, k, v host -> device
+ * staging buffers, runs attn_fwd, copies o (and lse when both lse pointers are
+ * non-null) back, all queued on `stream`; the caller synchronises the stream before
+ * reading o_host / lse_host.  Host buffers should be page-locked for the copies to
+ * be asynchronous.  The staging buffers (q_dev ... lse_dev) are caller-allocated
+ * device memory with the shapes and alignment attn_fwd requires.
+ */
+int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                  void *o_host, float *lse_host,
+                  void *q_dev, void *k_dev, void *v_dev, void *o_dev, float *lse_dev,
+                  int B, int H, int Sq, int Sk, int D, int causal, float scale,
+                  int dtype, attn_stream_t stream);
+
+/*
+ * attn_fwd_status -- synchronise `stream`, copy the current device's status word
+ * into *device_status (0, or the first ATTN_ERR_* a kernel recorded since the last
+ * read) and reset it to 0.  Returns ATTN_OK, ATTN_ERR_NULLPTR or ATTN_ERR_LAUNCH.
+ */
+int attn_fwd_status(attn_stream_t stream, int *device_status);
+
+/* Static string naming an ATTN_* code (never NULL). */
+const char *attn_fwd_strerror(int code);
+
+/* ABI version of this header, currently 1. */
+int attn_fwd_abi_version(void);
+
+/*
+ * attn_fwd_debug -- attn_fwd with kernel debug flags, for the tests.  Flag 1 makes
+ * the TMA producer skip the Q load so the MMA warp's first wait runs out: the call
+ * must end with ATTN_ERR_TIMEOUT in the status word, not hang.  Flag 0 is attn_fwd.
+ */
+int attn_fwd_debug(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int H, int Sq, int Sk, int D, int causal, float scale,
+                   int dtype, attn_stream_t stream, unsigned flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_FWD_H */

@@ -1,0 +1,113 @@
+"""CUDA path vs the fp64 oracle on identical seeded inputs, element by element
+(max |dO| <= 2e-2, max |dLSE| <= 1e-3), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import attention_forward_18_b200 as af
+import oracle
+from parity import O_TOL, LSE_TOL, check_full, compare, run_gpu
+from workloads import WORKLOADS, make_inputs, make_qkv, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_workload_whole(causal):
+    w = WORKLOADS["C1"]
+    check_full(w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, causal, w.seed)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bench_workload_whole(causal):
+    """The benchmark's workload (B=4, H=16, S=1024, D=64, fp16), every element."""
+    w = WORKLOADS["C2"]
+    check_full(w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, causal, w.seed)
+
+
+RAGGED = [(1, 1), (17, 17), (127, 127), (129, 129), (1000, 1000), (17, 300),
+          (300, 17), (129, 1000), (1000, 129), (255, 256), (256, 255), (384, 384)]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Sq,Sk", RAGGED)
+def test_ragged_shapes(Sq, Sk, causal, dtype, D):
+    check_full(2, 3, Sq, Sk, D, dtype, causal, seed=Sq * 7 + Sk)
+
+
+@pytest.mark.parametrize("name", ["C3", "C4", "C5"])
+def test_large_workloads_sampled_rows(name):
+    """Full-size workloads in the benchmark's launch configuration; sampled rows
+    (edges, every tile boundary of one head, random rows) against the oracle row by
+    row, and at every position the properties that hold at any size."""
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    for causal in w.causal:
+        o, lse = run_gpu(q, k, v, causal, w.scale)
+        assert np.isfinite(o).all() and np.isfinite(lse).all()
+        # O is a convex combination of V rows: |O| <= max |V| per head and feature
+        vmax = v.abs().amax(dim=2).double().numpy()            # [B,H,D]
+        assert (np.abs(o) <= vmax[:, :, None, :] + O_TOL).all()
+        rows = sample_rows(w.B, w.H, w.Sq, 96, seed=w.seed)
+        ro, rl = oracle.attn_ref_rows(q.double().numpy(), k.double().numpy(),
+                                      v.double().numpy(), rows, causal, w.scale)
+        idx = tuple(np.array(rows).T)
+        compare(o[idx], lse[idx], ro, rl, f"{name} causal={causal}")
+
+
+def test_lse_pointer_may_be_null():
+    q, k, v = make_qkv(1, 2, 200, 200, 64, "f16", 11)
+    o, lse = run_gpu(q, k, v, True, 0.125, with_lse=False)
+    assert lse is None
+    o_ref, _ = oracle.attn_ref(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                               True, 0.125)
+    assert np.abs(o - o_ref).max() <= O_TOL
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.3, 1.7])
+def test_unusual_scales(scale):
+    check_full(1, 2, 130, 260, 64, "bf16", True, seed=5, scale=scale)
+    check_full(1, 2, 130, 260, 128, "f16", False, seed=6, scale=scale)
+
+
+def test_deterministic_and_stream():
+    """Bitwise-identical results over repeated runs, also on a non-default stream."""
+    q, k, v = (t.cuda() for t in make_qkv(2, 4, 700, 900, 128, "bf16", 12))
+    o1, l1 = af.attention(q, k, v, causal=True)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o2, l2 = af.attention(q, k, v, causal=True, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    for _ in range(3):
+        o3, l3 = af.attention(q, k, v, causal=True)
+        assert torch.equal(o1, o3) and torch.equal(l1, l3)
+    assert af.attn_fwd_status() == 0
+
+
+def test_single_head_and_constant_value():
+    """B*H = 1; a constant V returns that constant (exactly representable)."""
+    q, k, _ = make_qkv(1, 1, 333, 333, 64, "f16", 13)
+    v = torch.full((1, 1, 333, 64), 0.75, dtype=torch.float16)
+    o, lse = run_gpu(q, k, v, False, 0.125)
+    assert np.abs(o - 0.75).max() <= 1e-3
+
+
+def test_host_buffers_entry_point():
+    """attn_fwd_host: pinned host in, host out, same numbers as the device call."""
+    B, H, S, D = 2, 2, 300, 128
+    q, k, v = make_qkv(B, H, S, S, D, "bf16", 14)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((B, H, S), dtype=torch.float32).pin_memory()
+    staging = (torch.empty_like(q, device="cuda"), torch.empty_like(k, device="cuda"),
+               torch.empty_like(v, device="cuda"), torch.empty_like(q, device="cuda"),
+               torch.empty((B, H, S), dtype=torch.float32, device="cuda"))
+    af.attention_host(qh, kh, vh, staging, causal=True, out=oh, lse=lh)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attn_ref(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                   True, 1 / np.sqrt(D))
+    compare(oh.double().numpy(), lh.double().numpy(), o_ref, l_ref, "host entry")
