@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--profile-once", action="store_true",
+                    help="launch each pass of the workload once and exit (for ncu captures)")
     return ap.parse_args()
 
 
@@ -440,10 +442,28 @@ def reference_arm(args, world, rank):
     }
 
 
+def profile_once(args):
+    """One launch per pass of the workload, nothing else on the GPU before it except
+    the input copies (a short, self-ending command for ncu)."""
+    import attention_forward_18_b200 as af
+    w = WORKLOADS[args.workload]
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    for c in w.causal:
+        af.attention(q, k, v, causal=c, scale=w.scale)
+    torch.cuda.synchronize()
+    status = af.attn_fwd_status()
+    if status != 0:
+        raise af.AttnError(status, "device status")
+    print(json.dumps({"profile_once": w.name, "passes": list(w.causal)}))
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup()
     try:
+        if args.profile_once:
+            profile_once(args)
+            return
         if args.impl == "reference":
             if rank == 0:
                 print(json.dumps(reference_arm(args, 1, rank)), flush=True)
