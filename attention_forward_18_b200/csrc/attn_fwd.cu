@@ -94,8 +94,8 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     if (Sq > kMaxSeq || Sk > kMaxSeq) return ATTN_ERR_SHAPE;
     const int64_t bh = static_cast<int64_t>(B) * H;
     if (bh > kMaxHeads) return ATTN_ERR_SHAPE;
-    const int64_t n_qb = (Sq + attn::BM - 1) / attn::BM;
-    if (n_qb * bh > INT_MAX) return ATTN_ERR_SHAPE;
+    const int64_t n_qp = (Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    if (n_qp * bh > INT_MAX) return ATTN_ERR_SHAPE;
     if (!std::isfinite(scale)) return ATTN_ERR_SCALE;
     auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
     if (mis16(q) || mis16(k) || mis16(v) || mis16(o)) return ATTN_ERR_ALIGN;
@@ -137,10 +137,9 @@ int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-// Ring depth: as many K/V stages as fit beside the Q tile while keeping the
-// shared-memory request above half an SM (one CTA per SM).
+// Ring depth: as many K/V stages as fit beside the two Q tiles in shared memory.
 template <int D>
-constexpr int kStages = (D == 64) ? 4 : 2;
+constexpr int kStages = (D == 64) ? 5 : 2;
 
 template <int D, bool BF16>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -168,10 +167,10 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     p.Sq = Sq;
     p.Sk = Sk;
     p.BH = BH;
-    p.n_qb = (Sq + attn::BM - 1) / attn::BM;
+    p.n_qp = (Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
     p.flags = flags;
-    const int grid = p.n_qb * BH;
+    const int grid = p.n_qp * BH;
     const bool c = causal != 0;
     if (D == 64) return bf16 ? launch_d<64, true>(tq, tk, tv, p, grid, c, stream)
                              : launch_d<64, false>(tq, tk, tv, p, grid, c, stream);

@@ -8,24 +8,34 @@
 // tensor-core matrix products; comrad404.com "Финал": parallel over heads with
 // sequential reads from HBM).
 //
-// One CTA owns one 128-row query tile of one (batch, head) and streams the head's
-// K/V in 128-key tiles:
-//   warp 0      TMA producer: Q once, then K_j / V_j into a ring of NS stages
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T (smem x smem -> TMEM) and
-//               O += P_j V_j (P from TMEM, V from smem -> TMEM)
-//   warp 2      owns the tensor-memory allocation
-//   warps 4..7  softmax: thread t owns query row t of the tile; reads S_j from TMEM,
-//               masks, updates the running max / normaliser, writes P_j (16-bit)
-//               over S_j in TMEM, rescales O in TMEM when the max moved by more
-//               than 2^8, and finally writes O / l and the LSE.
-// Tensor memory (512 columns): S/P double buffer at columns 0 and 128, O at 256.
-// Shared memory: Q tile + NS K tiles + NS V tiles, each tile 128 rows x D stored
-// as D/64 column chunks of 128 rows x 128 bytes in the 128-byte swizzle that TMA
-// writes and the tcgen05 descriptors read.
+// Work unit: one CTA owns two 128-row query tiles (rows q0 .. q0+255) of one
+// (batch, head) and streams that head's K/V in 128-key tiles; both query tiles share
+// every K/V tile brought into shared memory.
 //
-// Every mbarrier wait is bounded (WAIT_LIMIT_NS); on expiry the waiting role
-// records ATTN_ERR_TIMEOUT in the device status word, flags the CTA, and every role
-// leaves its loop, waits (again bounded) for its copies / MMAs in flight, and the
+//   warps 0-3   softmax of query tile 0 (thread t owns row t of the tile)
+//   warps 4-7   softmax of query tile 1
+//   warps 8-11  correction (rescale O in TMEM when a row max moved) and epilogue
+//   warp 12     MMA issuer (one thread)
+//   warp 13     TMA producer (one thread)
+//   warp 14     owns the tensor-memory allocation
+//   warp 15     idle
+//
+// Tensor memory (512 columns): S_0 at 0, S_1 at 128 (fp32 scores, then the 16-bit
+// probabilities P_t written over the first 64 columns), O_0 at 256, O_1 at 256 + D.
+// The MMA thread ping-pongs the two tiles so one tile's softmax overlaps the other
+// tile's matrix products:
+//     S_0,0  S_1,0 | PV_0,0  S_0,1 | PV_1,0  S_1,1 | PV_0,1  S_0,2 | ...
+// Shared memory: Q_0, Q_1 and an NS-stage ring of K and of V tiles; each tile is
+// 128 rows x D stored as D/64 column chunks of 128 rows x 128 bytes in the 128-byte
+// swizzle that TMA writes and the tcgen05 smem descriptors read.
+//
+// Registers: 512 threads launch with 128 registers each; setmaxnreg moves them to
+// 192 for the softmax warpgroups, 72 for the correction warpgroup and 56 for the
+// MMA / TMA / allocator warps (2*128*192 + 128*72 + 128*56 = 65536).
+//
+// Every mbarrier wait is bounded (WAIT_LIMIT_NS); on expiry the waiting role records
+// ATTN_ERR_TIMEOUT in the device status word and flags the CTA; every role then
+// leaves its loop, waits (again bounded) for the copies / MMAs it started, and the
 // CTA frees its tensor memory and exits.
 #pragma once
 
@@ -38,31 +48,31 @@ namespace attn {
 
 constexpr int BM = 128;                 // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;                 // keys per tile
+constexpr int ROWS_PER_CTA = 2 * BM;    // two query tiles per CTA
 constexpr int CHUNK_ELEMS = 64;         // 16-bit elements per 128-byte swizzle row
 constexpr int CHUNK_BYTES = 128 * 128;  // one chunk: 128 rows x 128 bytes
-constexpr int NUM_THREADS = 256;
+constexpr int NUM_THREADS = 512;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_S0 = 0;
-constexpr uint32_t TMEM_S1 = 128;
-constexpr uint32_t TMEM_O = 256;
-// Lazy rescaling: the running max used for the exponentials is only moved when a
-// row's new max exceeds it by more than this (log2 units); until then P can reach
-// 2^8, which fp16/bf16 hold exactly in range, and O and l stay consistent because
-// both are accumulated relative to the same stale max.
+constexpr uint32_t TMEM_S = 0;          // + 128 * tile
+constexpr uint32_t TMEM_O = 256;        // + D * tile
+// Lazy rescaling: the running max used for the exponentials only moves when a row's
+// new max exceeds it by more than this (log2 units).  Until then P can reach 2^8,
+// well inside fp16/bf16 range, and O and l stay consistent because both accumulate
+// relative to the same (stale) max, so O / l is unchanged.
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;   // 0.5 s per drain wait
 
 constexpr int STATUS_TIMEOUT = -8;  // ATTN_ERR_TIMEOUT
 
-// Bit 0: the producer never issues the Q load, so the MMA warp's first wait runs
+// Bit 0: the producer never issues the Q loads, so the MMA thread's first wait runs
 // out; only the timeout test sets it.
 constexpr uint32_t FLAG_SKIP_Q_LOAD = 1u;
 
 struct Params {
     void* o;            // [BH, Sq, D] 16-bit
     float* lse;         // [BH, Sq] fp32, may be null
-    int Sq, Sk, BH, n_qb;
+    int Sq, Sk, BH, n_qp;
     float scale_log2;   // scale * log2(e)
     uint32_t flags;
 };
@@ -72,13 +82,16 @@ struct SmemLayout {
     static_assert(D % CHUNK_ELEMS == 0, "head dim must be a multiple of 64");
     static constexpr int NCH = D / CHUNK_ELEMS;
     static constexpr int TILE_BYTES = NCH * CHUNK_BYTES;  // 128 rows x D x 2 bytes
-    static constexpr int Q_OFF = 0;
-    static constexpr int K_OFF = Q_OFF + TILE_BYTES;
+    static constexpr int Q_OFF = 0;                        // two query tiles
+    static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
     static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
-    static constexpr int BAR_OFF = V_OFF + NS * TILE_BYTES;
-    // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-    // p_full[2], o_done, drain
-    static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 1;
+    static constexpr int ALPHA_OFF = V_OFF + NS * TILE_BYTES;  // float [2][128]
+    static constexpr int FM_OFF = ALPHA_OFF + 2 * BM * 4;      // final max  [2][128]
+    static constexpr int FL_OFF = FM_OFF + 2 * BM * 4;         // final sum  [2][128]
+    static constexpr int BAR_OFF = FL_OFF + 2 * BM * 4;
+    // q_full[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
+    // p_full[2], o_done[2], o_ready[2], final[2], drain
+    static constexpr int NBAR = 2 + 4 * NS + 2 * 5 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, error flag
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1024
@@ -136,6 +149,101 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     else return ptx::pack_f16x2(lo, hi);
 }
 
+// Number of 128-key tiles query tile `t` of the CTA at row q0 needs (0 when the tile
+// lies past Sq).  Causal: keys up to the tile's last valid row (top-left mask).
+template <bool CAUSAL>
+__device__ __forceinline__ int kv_tiles_for(int q0, int t, int Sq, int Sk) {
+    const int first = q0 + BM * t;
+    if (first >= Sq) return 0;
+    const int n_all = (Sk + BN - 1) / BN;
+    if (!CAUSAL) return n_all;
+    const int last_row = min(first + BM - 1, Sq - 1);
+    return min(n_all, last_row / BN + 1);
+}
+
+// --------------------------------------------------------------------------- softmax
+// One KV tile of one query row held by this thread: read S from TMEM, mask, update
+// the running max (lazy), exponentiate, accumulate the normaliser, write P over S.
+// Returns alpha, the factor O must be multiplied by before P V is added (1 = none).
+template <bool IS_BF16, bool CAUSAL>
+__device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int qrow,
+                                              int q0t, float c_l2, float& m_used, float& l) {
+    uint32_t s[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        ptx::tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+    ptx::tmem_wait_ld();
+
+    // Keys past `lim` (tile-relative) are invisible: past Sk, or (causal) past qrow.
+    const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > q0t);
+    int lim = Sk - 1 - kv0;
+    if (CAUSAL) lim = min(lim, qrow - kv0);
+    const bool pos = c_l2 >= 0.f;
+    // row extreme of the raw scores: max for a positive scale, min for a negative one
+    float mt;
+    if (!need_mask) {
+        float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
+        if (pos) {
+#pragma unroll
+            for (int c = 2; c < 128; c += 2) {
+                a0 = fmaxf(a0, __uint_as_float(s[c]));
+                a1 = fmaxf(a1, __uint_as_float(s[c + 1]));
+            }
+            mt = fmaxf(a0, a1);
+        } else {
+#pragma unroll
+            for (int c = 2; c < 128; c += 2) {
+                a0 = fminf(a0, __uint_as_float(s[c]));
+                a1 = fminf(a1, __uint_as_float(s[c + 1]));
+            }
+            mt = fminf(a0, a1);
+        }
+    } else {
+        const uint32_t neutral = __float_as_uint(pos ? -INFINITY : INFINITY);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+            if (c > lim) s[c] = neutral;
+        float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
+#pragma unroll
+        for (int c = 2; c < 128; c += 2) {
+            a0 = pos ? fmaxf(a0, __uint_as_float(s[c])) : fminf(a0, __uint_as_float(s[c]));
+            a1 = pos ? fmaxf(a1, __uint_as_float(s[c + 1]))
+                     : fminf(a1, __uint_as_float(s[c + 1]));
+        }
+        mt = pos ? fmaxf(a0, a1) : fminf(a0, a1);
+    }
+    // every processed tile has a visible key in every row, so mt is finite here
+    const float m_tile = mt * c_l2;
+    float alpha = 1.f;
+    if (j == 0) {
+        m_used = m_tile;
+    } else if (m_tile > m_used + LAZY_RESCALE_LOG2) {
+        alpha = ptx::ex2(m_used - m_tile);
+        m_used = m_tile;
+    }
+    const float neg_m = -m_used;
+
+    // p = 2^(s * c - m): scale and shift in one fma, exponent on the SFU
+    float sum0 = 0.f, sum1 = 0.f;
+    uint32_t pk[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+        float p0 = ptx::ex2(fmaf(__uint_as_float(s[2 * c]), c_l2, neg_m));
+        float p1 = ptx::ex2(fmaf(__uint_as_float(s[2 * c + 1]), c_l2, neg_m));
+        if (need_mask) {
+            p0 = (2 * c > lim) ? 0.f : p0;
+            p1 = (2 * c + 1 > lim) ? 0.f : p1;
+        }
+        sum0 += p0;
+        sum1 += p1;
+        pk[c] = pack2<IS_BF16>(p0, p1);
+    }
+    l = l * alpha + (sum0 + sum1);
+    ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+    ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+    return alpha;
+}
+
 template <int D, int NS, bool IS_BF16, bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -153,60 +261,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t sQ = sbase + L::Q_OFF;
     const uint32_t sK = sbase + L::K_OFF;
     const uint32_t sV = sbase + L::V_OFF;
+    float* s_alpha = reinterpret_cast<float*>(smem + L::ALPHA_OFF);
+    float* s_fm = reinterpret_cast<float*>(smem + L::FM_OFF);
+    float* s_fl = reinterpret_cast<float*>(smem + L::FL_OFF);
     const uint32_t bars = sbase + L::BAR_OFF;
-    const uint32_t B_Q = bars;
-    auto B_KF = [&](int s) { return bars + 8u * (1 + s); };
-    auto B_KE = [&](int s) { return bars + 8u * (1 + NS + s); };
-    auto B_VF = [&](int s) { return bars + 8u * (1 + 2 * NS + s); };
-    auto B_VE = [&](int s) { return bars + 8u * (1 + 3 * NS + s); };
-    auto B_SF = [&](int b) { return bars + 8u * (1 + 4 * NS + b); };
-    auto B_PF = [&](int b) { return bars + 8u * (3 + 4 * NS + b); };
-    const uint32_t B_OD = bars + 8u * (5 + 4 * NS);
-    const uint32_t B_DR = bars + 8u * (6 + 4 * NS);
+    auto B_QF = [&](int t) { return bars + 8u * t; };
+    auto B_KF = [&](int s) { return bars + 8u * (2 + s); };
+    auto B_KE = [&](int s) { return bars + 8u * (2 + NS + s); };
+    auto B_VF = [&](int s) { return bars + 8u * (2 + 2 * NS + s); };
+    auto B_VE = [&](int s) { return bars + 8u * (2 + 3 * NS + s); };
+    auto B_SF = [&](int t) { return bars + 8u * (2 + 4 * NS + t); };
+    auto B_PF = [&](int t) { return bars + 8u * (4 + 4 * NS + t); };
+    auto B_OD = [&](int t) { return bars + 8u * (6 + 4 * NS + t); };
+    auto B_OR = [&](int t) { return bars + 8u * (8 + 4 * NS + t); };
+    auto B_FN = [&](int t) { return bars + 8u * (10 + 4 * NS + t); };
+    const uint32_t B_DR = bars + 8u * (12 + 4 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     Ctx ctx{reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4)};
 
-    // ---- which tile: causal grids go heaviest query block first
-    int qb, bh;
+    // ---- which rows: causal grids go heaviest query block first
+    int qp, bh;
     if constexpr (CAUSAL) {
-        qb = p.n_qb - 1 - static_cast<int>(blockIdx.x) / p.BH;
+        qp = p.n_qp - 1 - static_cast<int>(blockIdx.x) / p.BH;
         bh = static_cast<int>(blockIdx.x) % p.BH;
     } else {
-        qb = static_cast<int>(blockIdx.x) % p.n_qb;
-        bh = static_cast<int>(blockIdx.x) / p.n_qb;
+        qp = static_cast<int>(blockIdx.x) % p.n_qp;
+        bh = static_cast<int>(blockIdx.x) / p.n_qp;
     }
-    const int q0 = qb * BM;
-    const int n_kv_all = (p.Sk + BN - 1) / BN;
-    int n_kv = n_kv_all;
-    if constexpr (CAUSAL) {
-        const int last_row = min(q0 + BM - 1, p.Sq - 1);
-        n_kv = min(n_kv_all, last_row / BN + 1);
-    }
+    const int q0 = qp * ROWS_PER_CTA;
+    const int n_t0 = kv_tiles_for<CAUSAL>(q0, 0, p.Sq, p.Sk);
+    const int n_t1 = kv_tiles_for<CAUSAL>(q0, 1, p.Sq, p.Sk);
+    const int n_max = max(n_t0, n_t1);
 
     // ---- set-up
     if (threadIdx.x == 0) {
-        ptx::mbar_init(B_Q, 1);
+        for (int t = 0; t < 2; ++t) {
+            ptx::mbar_init(B_QF(t), 1);
+            ptx::mbar_init(B_SF(t), 1);
+            ptx::mbar_init(B_PF(t), BM);  // every softmax thread of the tile
+            ptx::mbar_init(B_OD(t), 1);
+            ptx::mbar_init(B_OR(t), BM);  // every correction thread
+            ptx::mbar_init(B_FN(t), BM);  // every softmax thread of the tile
+        }
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(B_KF(s), 1);
             ptx::mbar_init(B_KE(s), 1);
             ptx::mbar_init(B_VF(s), 1);
             ptx::mbar_init(B_VE(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(B_SF(b), 1);
-            ptx::mbar_init(B_PF(b), 4);  // one arrival per softmax warp
-        }
-        ptx::mbar_init(B_OD, 1);
         ptx::mbar_init(B_DR, 1);
         *ctx.err = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == 13 && lane == 0) {
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
     }
-    if (warp == 2) {
+    if (warp == 14) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
         ptx::tmem_relinquish();
     }
@@ -215,183 +327,87 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ================================================================ producer
-        if (lane == 0) {
-            const bool load_q = !(p.flags & FLAG_SKIP_Q_LOAD);
-            if (load_q) {
-                ptx::mbar_arrive_expect_tx(B_Q, L::TILE_BYTES);
-                for (int c = 0; c < L::NCH; ++c)
-                    ptx::tma_load_3d(sQ + c * CHUNK_BYTES, &tm_q, B_Q, c * CHUNK_ELEMS, q0, bh);
-            }
-            int last_k = -1, last_v = -1;  // last issued tile index
-            for (int j = 0; j < n_kv; ++j) {
-                const int s = j % NS;
-                const uint32_t ph = (j / NS) & 1;
-                if (!wait_bounded(ctx, B_KE(s), ph ^ 1)) break;
-                ptx::mbar_arrive_expect_tx(B_KF(s), L::TILE_BYTES);
-                for (int c = 0; c < L::NCH; ++c)
-                    ptx::tma_load_3d(sK + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_k, B_KF(s),
-                                     c * CHUNK_ELEMS, j * BN, bh);
-                last_k = j;
-                if (!wait_bounded(ctx, B_VE(s), ph ^ 1)) break;
-                ptx::mbar_arrive_expect_tx(B_VF(s), L::TILE_BYTES);
-                for (int c = 0; c < L::NCH; ++c)
-                    ptx::tma_load_3d(sV + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_v, B_VF(s),
-                                     c * CHUNK_ELEMS, j * BN, bh);
-                last_v = j;
-            }
-            // Let every copy this thread started land before the CTA can exit.
-            if (load_q) wait_drain(B_Q, 0);
-            for (int j = (last_k - NS + 1 > 0 ? last_k - NS + 1 : 0); j <= last_k; ++j)
-                wait_drain(B_KF(j % NS), (j / NS) & 1);
-            for (int j = (last_v - NS + 1 > 0 ? last_v - NS + 1 : 0); j <= last_v; ++j)
-                wait_drain(B_VF(j % NS), (j / NS) & 1);
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ================================================================ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t fmt = IS_BF16 ? 1u : 0u;
-            constexpr uint32_t idesc_qk = ptx::idesc_f16(fmt, BM, BN, 0);
-            constexpr uint32_t idesc_pv = ptx::idesc_f16(fmt, BM, D, 1);
-            bool ok = wait_bounded(ctx, B_Q, 0);
-            if (ok) ptx::tc_fence_after();
-            for (int j = 0; ok && j <= n_kv; ++j) {
-                if (j < n_kv) {
-                    // S_j = Q K_j^T  (both operands K-major, 128-byte swizzle)
-                    const int s = j % NS;
-                    if (!(ok = wait_bounded(ctx, B_KF(s), (j / NS) & 1))) break;
-                    ptx::tc_fence_after();
-                    const uint32_t d_tmem = tmem + ((j & 1) ? TMEM_S1 : TMEM_S0);
-                    const uint32_t kt = sK + s * L::TILE_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * CHUNK_BYTES + (kk % 4) * 32;
-                        const uint64_t a = ptx::smem_desc_sw128(sQ + off, 16, 1024);
-                        const uint64_t b = ptx::smem_desc_sw128(kt + off, 16, 1024);
-                        ptx::mma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    ptx::mma_commit(B_SF(j & 1));
-                    ptx::mma_commit(B_KE(s));
-                }
-                if (j >= 1) {
-                    // O += P_{j-1} V_{j-1}  (P in TMEM, V MN-major in smem)
-                    const int jp = j - 1;
-                    const int s = jp % NS;
-                    if (!(ok = wait_bounded(ctx, B_PF(jp & 1), (jp >> 1) & 1))) break;
-                    if (!(ok = wait_bounded(ctx, B_VF(s), (jp / NS) & 1))) break;
-                    ptx::tc_fence_after();
-                    const uint32_t a_tmem = tmem + ((jp & 1) ? TMEM_S1 : TMEM_S0);
-                    const uint32_t vt = sV + s * L::TILE_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint64_t b = ptx::smem_desc_sw128(vt + kk * 2048, CHUNK_BYTES, 1024);
-                        ptx::mma_ts(tmem + TMEM_O, a_tmem + kk * 8, b, idesc_pv,
-                                    (jp > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    ptx::mma_commit(B_VE(s));
-                    ptx::mma_commit(B_OD);
-                }
-            }
-            // Every MMA issued above completes before the CTA frees tensor memory.
-            ptx::mma_commit(B_DR);
-            wait_drain(B_DR, 0);
-        }
-        __syncwarp();
-    } else if (warp >= 4) {
+    if (warp < 8) {
         // ================================================================ softmax
-        const int wq = warp - 4;  // this warp's TMEM lane quarter
+        ptx::setmaxnreg_inc<192>();
+        const int t = warp >> 2;                    // query tile
+        const int wq = warp & 3;                    // TMEM lane quarter
         const int row = wq * 32 + lane;
-        const int qrow = q0 + row;
-        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-        const float sl2 = p.scale_log2;
-        float m_used = -INFINITY;  // running max (log2 units) the exponentials use
-        float l = 0.f;             // running normaliser relative to m_used
+        const int q0t = q0 + BM * t;
+        const int qrow = q0t + row;
+        const int n_t = t == 0 ? n_t0 : n_t1;
+        const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + TMEM_S + 128u * t;
+        const float c_l2 = p.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
-            const int sb = j & 1;
-            if (!(ok = warp_wait(ctx, B_SF(sb), (j >> 1) & 1))) break;
+        for (int j = 0; j < n_t; ++j) {
+            if (!(ok = warp_wait(ctx, B_SF(t), j & 1))) break;
             ptx::tc_fence_after();
-            const uint32_t tS = tmem + lane_base + (sb ? TMEM_S1 : TMEM_S0);
-            uint32_t raw[4][32];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, raw[c]);
-            ptx::tmem_wait_ld();
-
-            float x[128];
-            const int kv0 = j * BN;
-            const bool need_mask = (kv0 + BN > p.Sk) || (CAUSAL && kv0 + BN - 1 > q0);
-            float mt = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                float t = __uint_as_float(raw[c >> 5][c & 31]) * sl2;
-                if (need_mask) {
-                    const int key = kv0 + c;
-                    if (key >= p.Sk || (CAUSAL && key > qrow)) t = -INFINITY;
-                }
-                x[c] = t;
-                mt = fmaxf(mt, t);
-            }
-            float alpha = 1.f;
-            bool rescale = false;
-            if (j == 0) {
-                m_used = mt;
-            } else if (mt > m_used + LAZY_RESCALE_LOG2) {
-                alpha = ptx::ex2(m_used - mt);
-                m_used = mt;
-                rescale = true;
-            }
-            float sum = 0.f;
-            uint32_t pk[64];
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float p0 = ptx::ex2(x[2 * c] - m_used);
-                const float p1 = ptx::ex2(x[2 * c + 1] - m_used);
-                sum += p0 + p1;
-                pk[c] = pack2<IS_BF16>(p0, p1);
-            }
-            l = l * alpha + sum;
-            // P_j over S_j: 128 16-bit values = 64 columns
-            ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-            ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-
-            if (j > 0) {
-                // O holds sum over tiles < j; PV_{j-1} must be done before touching it
-                if (!(ok = warp_wait(ctx, B_OD, (j - 1) & 1))) break;
-                ptx::tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t ov[32];
-                        const uint32_t tO = tmem + lane_base + TMEM_O + 32 * c;
-                        ptx::tmem_ld32(tO, ov);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                        ptx::tmem_st32(tO, ov);
-                    }
-                }
-            }
+            const float alpha =
+                softmax_tile<IS_BF16, CAUSAL>(tS, j, j * BN, p.Sk, qrow, q0t, c_l2, m_used, l);
+            s_alpha[t * BM + row] = alpha;
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(B_PF(sb));
+            ptx::mbar_arrive(B_PF(t));
         }
-
+        if (ok && n_t > 0) {
+            s_fm[t * BM + row] = m_used;
+            s_fl[t * BM + row] = l;
+            ptx::mbar_arrive(B_FN(t));
+        }
+    } else if (warp < 12) {
+        // ================================================================ correction
+        ptx::setmaxnreg_dec<72>();
+        const int wq = warp & 3;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        bool ok = true;
+        for (int j = 0; ok && j < n_max; ++j) {
+            for (int t = 0; t < 2; ++t) {
+                if (j >= (t == 0 ? n_t0 : n_t1)) continue;
+                if (!(ok = warp_wait(ctx, B_PF(t), j & 1))) break;  // alpha_j written
+                if (j > 0) {
+                    if (!(ok = warp_wait(ctx, B_OD(t), (j - 1) & 1))) break;  // PV_{j-1} done
+                    ptx::tc_fence_after();
+                    const float alpha = s_alpha[t * BM + row];
+                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                        const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t ov[32];
+                            ptx::tmem_ld32(tO + 32 * c, ov);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                            ptx::tmem_st32(tO + 32 * c, ov);
+                        }
+                        ptx::tmem_wait_st();
+                    }
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(B_OR(t));
+            }
+        }
         // ---- epilogue: O / l in fp32, one rounding to 16 bits; LSE in natural log
-        if (ok) ok = warp_wait(ctx, B_OD, (n_kv - 1) & 1);
-        if (ok) {
+        for (int t = 0; ok && t < 2; ++t) {
+            const int n_t = t == 0 ? n_t0 : n_t1;
+            if (n_t == 0) continue;
+            if (!(ok = warp_wait(ctx, B_FN(t), 0))) break;
+            if (!(ok = warp_wait(ctx, B_OD(t), (n_t - 1) & 1))) break;
             ptx::tc_fence_after();
+            const float m_used = s_fm[t * BM + row];
+            const float l = s_fl[t * BM + row];
             const float inv_l = 1.f / l;
+            const int qrow = q0 + BM * t + row;
             const bool store = qrow < p.Sq;
             uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
                              (static_cast<int64_t>(bh) * p.Sq + qrow) * D;
+            const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t ov[32];
-                ptx::tmem_ld32(tmem + lane_base + TMEM_O + 32 * c, ov);
+                ptx::tmem_ld32(tO + 32 * c, ov);
                 ptx::tmem_wait_ld();
                 uint32_t packed[16];
 #pragma unroll
@@ -410,12 +426,117 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 p.lse[static_cast<int64_t>(bh) * p.Sq + qrow] =
                     (m_used + log2f(l)) * 0.69314718055994530942f;
         }
+    } else {
+        ptx::setmaxnreg_dec<56>();
+        if (warp == 12) {
+            // ============================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t fmt = IS_BF16 ? 1u : 0u;
+                constexpr uint32_t idesc_qk = ptx::idesc_f16(fmt, BM, BN, 0);
+                constexpr uint32_t idesc_pv = ptx::idesc_f16(fmt, BM, D, 1);
+                const int n_t[2] = {n_t0, n_t1};
+                // S_t,j = Q_t K_j^T  (both operands K-major, 128-byte swizzle)
+                auto issue_s = [&](int t, int j) {
+                    const uint32_t qt = sQ + t * L::TILE_BYTES;
+                    const uint32_t kt = sK + (j % NS) * L::TILE_BYTES;
+                    const uint32_t d_tmem = tmem + TMEM_S + 128u * t;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * CHUNK_BYTES + (kk % 4) * 32;
+                        ptx::mma_ss(d_tmem, ptx::smem_desc_sw128(qt + off, 16, 1024),
+                                    ptx::smem_desc_sw128(kt + off, 16, 1024), idesc_qk,
+                                    kk > 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(B_SF(t));
+                };
+                // O_t += P_t,j V_j  (P from TMEM, V MN-major in smem)
+                auto issue_pv = [&](int t, int j) {
+                    const uint32_t vt = sV + (j % NS) * L::TILE_BYTES;
+                    const uint32_t a_tmem = tmem + TMEM_S + 128u * t;
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        ptx::mma_ts(tmem + TMEM_O + D * t, a_tmem + kk * 8,
+                                    ptx::smem_desc_sw128(vt + kk * 2048, CHUNK_BYTES, 1024),
+                                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_commit(B_OD(t));
+                };
+                bool ok = wait_bounded(ctx, B_QF(0), 0) && wait_bounded(ctx, B_QF(1), 0) &&
+                          wait_bounded(ctx, B_KF(0), 0);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    for (int t = 0; t < 2; ++t)
+                        if (n_t[t] > 0) issue_s(t, 0);
+                    ptx::mma_commit(B_KE(0));
+                }
+                for (int j = 0; ok && j < n_max; ++j) {
+                    const bool nxt = j + 1 < n_max;
+                    if (nxt && !(ok = wait_bounded(ctx, B_KF((j + 1) % NS), ((j + 1) / NS) & 1)))
+                        break;
+                    if (!(ok = wait_bounded(ctx, B_VF(j % NS), (j / NS) & 1))) break;
+                    for (int t = 0; t < 2; ++t) {
+                        if (j >= n_t[t]) continue;
+                        if (!(ok = wait_bounded(ctx, B_PF(t), j & 1))) break;
+                        if (!(ok = wait_bounded(ctx, B_OR(t), j & 1))) break;
+                        ptx::tc_fence_after();
+                        issue_pv(t, j);
+                        if (j + 1 < n_t[t]) issue_s(t, j + 1);
+                    }
+                    if (!ok) break;
+                    ptx::mma_commit(B_VE(j % NS));
+                    if (nxt) ptx::mma_commit(B_KE((j + 1) % NS));
+                }
+                // Every MMA issued above completes before the CTA frees tensor memory.
+                ptx::mma_commit(B_DR);
+                wait_drain(B_DR, 0);
+            }
+            __syncwarp();
+        } else if (warp == 13) {
+            // ============================================================ producer
+            if (lane == 0) {
+                const bool load_q = !(p.flags & FLAG_SKIP_Q_LOAD);
+                if (load_q) {
+                    for (int t = 0; t < 2; ++t) {
+                        ptx::mbar_arrive_expect_tx(B_QF(t), L::TILE_BYTES);
+                        for (int c = 0; c < L::NCH; ++c)
+                            ptx::tma_load_3d(sQ + t * L::TILE_BYTES + c * CHUNK_BYTES, &tm_q,
+                                             B_QF(t), c * CHUNK_ELEMS, q0 + BM * t, bh);
+                    }
+                }
+                int last_k = -1, last_v = -1;  // last issued tile index
+                for (int j = 0; j < n_max; ++j) {
+                    const int s = j % NS;
+                    const uint32_t ph = (j / NS) & 1;
+                    if (!wait_bounded(ctx, B_KE(s), ph ^ 1)) break;
+                    ptx::mbar_arrive_expect_tx(B_KF(s), L::TILE_BYTES);
+                    for (int c = 0; c < L::NCH; ++c)
+                        ptx::tma_load_3d(sK + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_k,
+                                         B_KF(s), c * CHUNK_ELEMS, j * BN, bh);
+                    last_k = j;
+                    if (!wait_bounded(ctx, B_VE(s), ph ^ 1)) break;
+                    ptx::mbar_arrive_expect_tx(B_VF(s), L::TILE_BYTES);
+                    for (int c = 0; c < L::NCH; ++c)
+                        ptx::tma_load_3d(sV + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_v,
+                                         B_VF(s), c * CHUNK_ELEMS, j * BN, bh);
+                    last_v = j;
+                }
+                // Let every copy this thread started land before the CTA can exit.
+                if (load_q) {
+                    wait_drain(B_QF(0), 0);
+                    wait_drain(B_QF(1), 0);
+                }
+                for (int j = (last_k - NS + 1 > 0 ? last_k - NS + 1 : 0); j <= last_k; ++j)
+                    wait_drain(B_KF(j % NS), (j / NS) & 1);
+                for (int j = (last_v - NS + 1 > 0 ? last_v - NS + 1 : 0); j <= last_v; ++j)
+                    wait_drain(B_VF(j % NS), (j / NS) & 1);
+            }
+            __syncwarp();
+        }
     }
 
     // ---- tear-down: every role is out of its loop; free tensor memory
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 14) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, TMEM_COLS);
     }
