@@ -12,9 +12,10 @@
 // (batch, head) and streams that head's K/V in 128-key tiles; both query tiles share
 // every K/V tile brought into shared memory.
 //
-//   warps 0-3   softmax of query tile 0 (thread t owns row t of the tile)
-//   warps 4-7   softmax of query tile 1
-//   warps 8-11  correction (rescale O in TMEM when a row max moved) and epilogue
+//   warps 0-3   softmax of query tile 0 (thread t owns row t of the tile); also
+//               rescales O_0 in TMEM on the rare KV tiles where a row max moved
+//   warps 4-7   softmax of query tile 1 (same for O_1)
+//   warps 8-11  epilogue: O / l, 16-bit rounding, stores of O and LSE
 //   warp 12     MMA issuer (one thread)
 //   warp 13     TMA producer (one thread)
 //   warp 14     owns the tensor-memory allocation
@@ -25,13 +26,16 @@
 // The MMA thread ping-pongs the two tiles so one tile's softmax overlaps the other
 // tile's matrix products:
 //     S_0,0  S_1,0 | PV_0,0  S_0,1 | PV_1,0  S_1,1 | PV_0,1  S_0,2 | ...
+// tcgen05 MMAs issued by one thread complete in issue order, so once S_t,j is
+// complete PV_t,j-1 is too and nothing touches O_t until P_t,j is handed over: the
+// softmax warps rescale O_t in place at that point, with no extra hand-off.
 // Shared memory: Q_0, Q_1 and an NS-stage ring of K and of V tiles; each tile is
 // 128 rows x D stored as D/64 column chunks of 128 rows x 128 bytes in the 128-byte
 // swizzle that TMA writes and the tcgen05 smem descriptors read.
 //
 // Registers: 512 threads launch with 128 registers each; setmaxnreg moves them to
-// 192 for the softmax warpgroups, 72 for the correction warpgroup and 56 for the
-// MMA / TMA / allocator warps (2*128*192 + 128*72 + 128*56 = 65536).
+// 192 for the softmax warpgroups, 64 for the epilogue warpgroup and 64 for the
+// MMA / TMA / allocator warps (2*128*192 + 128*64 + 128*64 = 65536).
 //
 // Every mbarrier wait is bounded (WAIT_LIMIT_NS); on expiry the waiting role records
 // ATTN_ERR_TIMEOUT in the device status word and flags the CTA; every role then
@@ -60,6 +64,13 @@ constexpr uint32_t TMEM_O = 256;        // + D * tile
 // well inside fp16/bf16 range, and O and l stay consistent because both accumulate
 // relative to the same (stale) max, so O / l is unchanged.
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;
+// 2^f on f in [-1/2, 1/2]: degree-3 polynomial with minimax relative error, fitted
+// by the Remez exchange in fit_exp2_poly.py (max relative error 7.5e-5 in fp32
+// evaluation, below the half-ulp of fp16 / bf16 the probabilities are rounded to).
+constexpr float EXP2_C0 = 0.9999280571937561f;
+constexpr float EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.2426111251115799f;
+constexpr float EXP2_C3 = 0.0551716685295105f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;   // 0.5 s per drain wait
 
@@ -85,13 +96,12 @@ struct SmemLayout {
     static constexpr int Q_OFF = 0;                        // two query tiles
     static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
     static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
-    static constexpr int ALPHA_OFF = V_OFF + NS * TILE_BYTES;  // float [2][128]
-    static constexpr int FM_OFF = ALPHA_OFF + 2 * BM * 4;      // final max  [2][128]
-    static constexpr int FL_OFF = FM_OFF + 2 * BM * 4;         // final sum  [2][128]
+    static constexpr int FM_OFF = V_OFF + NS * TILE_BYTES;  // final max  float [2][128]
+    static constexpr int FL_OFF = FM_OFF + 2 * BM * 4;      // final sum  float [2][128]
     static constexpr int BAR_OFF = FL_OFF + 2 * BM * 4;
     // q_full[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-    // p_full[2], o_done[2], o_ready[2], final[2], drain
-    static constexpr int NBAR = 2 + 4 * NS + 2 * 5 + 1;
+    // p_full[2], o_final[2], stats[2], drain
+    static constexpr int NBAR = 2 + 4 * NS + 2 * 4 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, error flag
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1024
@@ -162,55 +172,99 @@ __device__ __forceinline__ int kv_tiles_for(int q0, int t, int Sq, int Sk) {
 }
 
 // --------------------------------------------------------------------------- softmax
-// One KV tile of one query row held by this thread: read S from TMEM, mask, update
-// the running max (lazy), exponentiate, accumulate the normaliser, write P over S.
-// Returns alpha, the factor O must be multiplied by before P V is added (1 = none).
-template <bool IS_BF16, bool CAUSAL>
+// 2^x on the FMA pipe (x <= 2^7): n = round(x) by the 1.5*2^23 addition trick,
+// f = x - n, 2^f from the fitted polynomial, and n added to the exponent field.
+// Arguments below -125 are clamped (the result stays a normal number).
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    const float q = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, EXP2_C0);
+    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
+// Row extreme of 64 raw scores, folded into eight running accumulators: max for a
+// positive scale, min for a negative one (the extreme of scale * s).
+template <bool POS>
+__device__ __forceinline__ void extreme64(const uint32_t* s, float (&a)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+            const float x = __uint_as_float(s[i + 8 * k]);
+            const float y = __uint_as_float(s[i + 8 * k + 8]);
+            a[i] = POS ? ptx::max3(a[i], x, y) : ptx::min3(a[i], x, y);
+        }
+    }
+}
+
+template <bool POS>
+__device__ __forceinline__ float extreme128(uint32_t tS, uint32_t (&s)[128]) {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = POS ? -INFINITY : INFINITY;
+    // first half already loaded; the second half's load runs under the first's reduction
+    ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+    ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+    extreme64<POS>(&s[0], a);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+    extreme64<POS>(&s[64], a);
+    const float b0 = POS ? ptx::max3(a[0], a[1], a[2]) : ptx::min3(a[0], a[1], a[2]);
+    const float b1 = POS ? ptx::max3(a[3], a[4], a[5]) : ptx::min3(a[3], a[4], a[5]);
+    return POS ? ptx::max3(b0, b1, fmaxf(a[6], a[7])) : ptx::min3(b0, b1, fminf(a[6], a[7]));
+}
+
+// One KV tile of the query row this thread owns: read S_j from TMEM, mask, update the
+// running max (lazily), exponentiate, accumulate the normaliser and write P_j (16-bit)
+// over S_j.  Every POLY-th column pair takes the polynomial 2^x on the FMA pipe, the
+// rest the SFU's ex2 (0 = SFU only).  Returns alpha, the factor O must be scaled by
+// before P_j V_j is added (1 = none).
+template <bool IS_BF16, bool CAUSAL, int POLY>
 __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int qrow,
                                               int q0t, float c_l2, float& m_used, float& l) {
     uint32_t s[128];
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        ptx::tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+    ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
     ptx::tmem_wait_ld();
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
 
     // Keys past `lim` (tile-relative) are invisible: past Sk, or (causal) past qrow.
     const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > q0t);
     int lim = Sk - 1 - kv0;
     if (CAUSAL) lim = min(lim, qrow - kv0);
     const bool pos = c_l2 >= 0.f;
-    // row extreme of the raw scores: max for a positive scale, min for a negative one
-    float mt;
-    if (!need_mask) {
-        float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
-        if (pos) {
-#pragma unroll
-            for (int c = 2; c < 128; c += 2) {
-                a0 = fmaxf(a0, __uint_as_float(s[c]));
-                a1 = fmaxf(a1, __uint_as_float(s[c + 1]));
-            }
-            mt = fmaxf(a0, a1);
-        } else {
-#pragma unroll
-            for (int c = 2; c < 128; c += 2) {
-                a0 = fminf(a0, __uint_as_float(s[c]));
-                a1 = fminf(a1, __uint_as_float(s[c + 1]));
-            }
-            mt = fminf(a0, a1);
-        }
-    } else {
+    if (need_mask) {
+        // the second half is read here too, so the masking sees all 128 columns
+        ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        ptx::tmem_wait_ld();
+        ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
         const uint32_t neutral = __float_as_uint(pos ? -INFINITY : INFINITY);
 #pragma unroll
         for (int c = 0; c < 128; ++c)
             if (c > lim) s[c] = neutral;
-        float a0 = __uint_as_float(s[0]), a1 = __uint_as_float(s[1]);
+    }
+    float mt;
+    if (need_mask) {
+        float a[8];
 #pragma unroll
-        for (int c = 2; c < 128; c += 2) {
-            a0 = pos ? fmaxf(a0, __uint_as_float(s[c])) : fminf(a0, __uint_as_float(s[c]));
-            a1 = pos ? fmaxf(a1, __uint_as_float(s[c + 1]))
-                     : fminf(a1, __uint_as_float(s[c + 1]));
+        for (int i = 0; i < 8; ++i) a[i] = pos ? -INFINITY : INFINITY;
+        if (pos) {
+            extreme64<true>(&s[0], a);
+            extreme64<true>(&s[64], a);
+        } else {
+            extreme64<false>(&s[0], a);
+            extreme64<false>(&s[64], a);
         }
-        mt = pos ? fmaxf(a0, a1) : fminf(a0, a1);
+#pragma unroll
+        for (int i = 1; i < 8; ++i) a[0] = pos ? fmaxf(a[0], a[i]) : fminf(a[0], a[i]);
+        mt = a[0];
+    } else {
+        mt = pos ? extreme128<true>(tS, s) : extreme128<false>(tS, s);
     }
     // every processed tile has a visible key in every row, so mt is finite here
     const float m_tile = mt * c_l2;
@@ -223,13 +277,21 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     }
     const float neg_m = -m_used;
 
-    // p = 2^(s * c - m): scale and shift in one fma, exponent on the SFU
+    // p = 2^(s * c - m): scale and shift in one fma
     float sum0 = 0.f, sum1 = 0.f;
     uint32_t pk[64];
 #pragma unroll
     for (int c = 0; c < 64; ++c) {
-        float p0 = ptx::ex2(fmaf(__uint_as_float(s[2 * c]), c_l2, neg_m));
-        float p1 = ptx::ex2(fmaf(__uint_as_float(s[2 * c + 1]), c_l2, neg_m));
+        const float x0 = fmaf(__uint_as_float(s[2 * c]), c_l2, neg_m);
+        const float x1 = fmaf(__uint_as_float(s[2 * c + 1]), c_l2, neg_m);
+        float p0, p1;
+        if (POLY > 0 && (c % POLY) == POLY - 1) {
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+        } else {
+            p0 = ptx::ex2(x0);
+            p1 = ptx::ex2(x1);
+        }
         if (need_mask) {
             p0 = (2 * c > lim) ? 0.f : p0;
             p1 = (2 * c + 1 > lim) ? 0.f : p1;
@@ -243,6 +305,12 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
     return alpha;
 }
+
+// Exponent split between the SFU and the FMA pipe: every kPolyEvery-th column pair
+// takes the polynomial.  (On B200 the split changes the time by a few percent either
+// way; it also keeps the softmax within its 192 registers.)
+template <int D>
+constexpr int kPolyEvery = (D == 64) ? 2 : 4;
 
 template <int D, int NS, bool IS_BF16, bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -261,7 +329,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t sQ = sbase + L::Q_OFF;
     const uint32_t sK = sbase + L::K_OFF;
     const uint32_t sV = sbase + L::V_OFF;
-    float* s_alpha = reinterpret_cast<float*>(smem + L::ALPHA_OFF);
     float* s_fm = reinterpret_cast<float*>(smem + L::FM_OFF);
     float* s_fl = reinterpret_cast<float*>(smem + L::FL_OFF);
     const uint32_t bars = sbase + L::BAR_OFF;
@@ -270,12 +337,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto B_KE = [&](int s) { return bars + 8u * (2 + NS + s); };
     auto B_VF = [&](int s) { return bars + 8u * (2 + 2 * NS + s); };
     auto B_VE = [&](int s) { return bars + 8u * (2 + 3 * NS + s); };
-    auto B_SF = [&](int t) { return bars + 8u * (2 + 4 * NS + t); };
-    auto B_PF = [&](int t) { return bars + 8u * (4 + 4 * NS + t); };
-    auto B_OD = [&](int t) { return bars + 8u * (6 + 4 * NS + t); };
-    auto B_OR = [&](int t) { return bars + 8u * (8 + 4 * NS + t); };
-    auto B_FN = [&](int t) { return bars + 8u * (10 + 4 * NS + t); };
-    const uint32_t B_DR = bars + 8u * (12 + 4 * NS);
+    auto B_SF = [&](int t) { return bars + 8u * (2 + 4 * NS + t); };   // S_t,j in TMEM
+    auto B_PF = [&](int t) { return bars + 8u * (4 + 4 * NS + t); };   // P_t,j (+ O_t) ready
+    auto B_OF = [&](int t) { return bars + 8u * (6 + 4 * NS + t); };   // last PV_t done
+    auto B_ST = [&](int t) { return bars + 8u * (8 + 4 * NS + t); };   // final m, l in smem
+    const uint32_t B_DR = bars + 8u * (10 + 4 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     Ctx ctx{reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4)};
 
@@ -298,10 +364,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(B_QF(t), 1);
             ptx::mbar_init(B_SF(t), 1);
-            ptx::mbar_init(B_PF(t), BM);  // every softmax thread of the tile
-            ptx::mbar_init(B_OD(t), 1);
-            ptx::mbar_init(B_OR(t), BM);  // every correction thread
-            ptx::mbar_init(B_FN(t), BM);  // every softmax thread of the tile
+            ptx::mbar_init(B_PF(t), 4);  // one arrival per softmax warp
+            ptx::mbar_init(B_OF(t), 1);
+            ptx::mbar_init(B_ST(t), 4);  // one arrival per softmax warp
         }
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(B_KF(s), 1);
@@ -336,65 +401,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int q0t = q0 + BM * t;
         const int qrow = q0t + row;
         const int n_t = t == 0 ? n_t0 : n_t1;
-        const uint32_t tS = tmem + (static_cast<uint32_t>(wq * 32) << 16) + TMEM_S + 128u * t;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_base + TMEM_S + 128u * t;
+        const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
         const float c_l2 = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_t; ++j) {
             if (!(ok = warp_wait(ctx, B_SF(t), j & 1))) break;
             ptx::tc_fence_after();
-            const float alpha =
-                softmax_tile<IS_BF16, CAUSAL>(tS, j, j * BN, p.Sk, qrow, q0t, c_l2, m_used, l);
-            s_alpha[t * BM + row] = alpha;
+            const float alpha = softmax_tile<IS_BF16, CAUSAL, kPolyEvery<D>>(
+                tS, j, j * BN, p.Sk, qrow, q0t, c_l2, m_used, l);
+            // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
+            // bring it to the new max before PV_t,j adds to it
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t ov[32];
+                    ptx::tmem_ld32(tO + 32 * c, ov);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence32(ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                    ptx::tmem_st32(tO + 32 * c, ov);
+                }
+            }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
-            ptx::mbar_arrive(B_PF(t));
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(B_PF(t));
         }
         if (ok && n_t > 0) {
             s_fm[t * BM + row] = m_used;
             s_fl[t * BM + row] = l;
-            ptx::mbar_arrive(B_FN(t));
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(B_ST(t));
         }
     } else if (warp < 12) {
-        // ================================================================ correction
-        ptx::setmaxnreg_dec<72>();
+        // ================================================================ epilogue
+        ptx::setmaxnreg_dec<64>();
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         bool ok = true;
-        for (int j = 0; ok && j < n_max; ++j) {
-            for (int t = 0; t < 2; ++t) {
-                if (j >= (t == 0 ? n_t0 : n_t1)) continue;
-                if (!(ok = warp_wait(ctx, B_PF(t), j & 1))) break;  // alpha_j written
-                if (j > 0) {
-                    if (!(ok = warp_wait(ctx, B_OD(t), (j - 1) & 1))) break;  // PV_{j-1} done
-                    ptx::tc_fence_after();
-                    const float alpha = s_alpha[t * BM + row];
-                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                        const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
-#pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t ov[32];
-                            ptx::tmem_ld32(tO + 32 * c, ov);
-                            ptx::tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                            ptx::tmem_st32(tO + 32 * c, ov);
-                        }
-                        ptx::tmem_wait_st();
-                    }
-                }
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(B_OR(t));
-            }
-        }
-        // ---- epilogue: O / l in fp32, one rounding to 16 bits; LSE in natural log
+        // O / l in fp32, one rounding to 16 bits; LSE in natural log
         for (int t = 0; ok && t < 2; ++t) {
             const int n_t = t == 0 ? n_t0 : n_t1;
             if (n_t == 0) continue;
-            if (!(ok = warp_wait(ctx, B_FN(t), 0))) break;
-            if (!(ok = warp_wait(ctx, B_OD(t), (n_t - 1) & 1))) break;
+            if (!(ok = warp_wait(ctx, B_ST(t), 0))) break;
+            if (!(ok = warp_wait(ctx, B_OF(t), 0))) break;
             ptx::tc_fence_after();
             const float m_used = s_fm[t * BM + row];
             const float l = s_fl[t * BM + row];
@@ -409,6 +465,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint32_t ov[32];
                 ptx::tmem_ld32(tO + 32 * c, ov);
                 ptx::tmem_wait_ld();
+                ptx::reg_fence32(ov);
                 uint32_t packed[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -427,7 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     (m_used + log2f(l)) * 0.69314718055994530942f;
         }
     } else {
-        ptx::setmaxnreg_dec<56>();
+        ptx::setmaxnreg_dec<64>();
         if (warp == 12) {
             // ============================================================ MMA issuer
             if (lane == 0) {
@@ -435,30 +492,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 constexpr uint32_t idesc_qk = ptx::idesc_f16(fmt, BM, BN, 0);
                 constexpr uint32_t idesc_pv = ptx::idesc_f16(fmt, BM, D, 1);
                 const int n_t[2] = {n_t0, n_t1};
+                // Descriptors: the high word is common to every operand tile; per MMA only
+                // the start-address field of the low word moves, by a compile-time offset.
+                constexpr uint32_t desc_hi = ptx::smem_desc_hi_sw128(1024);
+                const uint32_t dq0 = ptx::smem_desc_lo(sQ, 16);
+                const uint32_t dk0 = ptx::smem_desc_lo(sK, 16);
+                const uint32_t dv0 = ptx::smem_desc_lo(sV, CHUNK_BYTES);
+                constexpr uint32_t TILE16 = L::TILE_BYTES >> 4;
                 // S_t,j = Q_t K_j^T  (both operands K-major, 128-byte swizzle)
                 auto issue_s = [&](int t, int j) {
-                    const uint32_t qt = sQ + t * L::TILE_BYTES;
-                    const uint32_t kt = sK + (j % NS) * L::TILE_BYTES;
+                    const uint32_t qd = dq0 + static_cast<uint32_t>(t) * TILE16;
+                    const uint32_t kd = dk0 + static_cast<uint32_t>(j % NS) * TILE16;
                     const uint32_t d_tmem = tmem + TMEM_S + 128u * t;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk / 4) * CHUNK_BYTES + (kk % 4) * 32;
-                        ptx::mma_ss(d_tmem, ptx::smem_desc_sw128(qt + off, 16, 1024),
-                                    ptx::smem_desc_sw128(kt + off, 16, 1024), idesc_qk,
-                                    kk > 0 ? 1u : 0u);
+                        const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
+                        ptx::mma_ss2(d_tmem, qd + off, kd + off, desc_hi, idesc_qk,
+                                     kk > 0 ? 1u : 0u);
                     }
                     ptx::mma_commit(B_SF(t));
                 };
                 // O_t += P_t,j V_j  (P from TMEM, V MN-major in smem)
                 auto issue_pv = [&](int t, int j) {
-                    const uint32_t vt = sV + (j % NS) * L::TILE_BYTES;
+                    const uint32_t vd = dv0 + static_cast<uint32_t>(j % NS) * TILE16;
                     const uint32_t a_tmem = tmem + TMEM_S + 128u * t;
+                    const uint32_t d_tmem = tmem + TMEM_O + D * t;
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk)
-                        ptx::mma_ts(tmem + TMEM_O + D * t, a_tmem + kk * 8,
-                                    ptx::smem_desc_sw128(vt + kk * 2048, CHUNK_BYTES, 1024),
-                                    idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit(B_OD(t));
+                        ptx::mma_ts2(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), desc_hi,
+                                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    if (j == n_t[t] - 1) ptx::mma_commit(B_OF(t));
                 };
                 bool ok = wait_bounded(ctx, B_QF(0), 0) && wait_bounded(ctx, B_QF(1), 0) &&
                           wait_bounded(ctx, B_KF(0), 0);
@@ -476,7 +539,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int t = 0; t < 2; ++t) {
                         if (j >= n_t[t]) continue;
                         if (!(ok = wait_bounded(ctx, B_PF(t), j & 1))) break;
-                        if (!(ok = wait_bounded(ctx, B_OR(t), j & 1))) break;
                         ptx::tc_fence_after();
                         issue_pv(t, j);
                         if (j + 1 < n_t[t]) issue_s(t, j + 1);
