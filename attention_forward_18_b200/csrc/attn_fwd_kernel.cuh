@@ -34,8 +34,8 @@
 // swizzle that TMA writes and the tcgen05 smem descriptors read.
 //
 // Registers: 512 threads launch with 128 registers each; setmaxnreg moves them to
-// 192 for the softmax warpgroups, 64 for the epilogue warpgroup and 64 for the
-// MMA / TMA / allocator warps (2*128*192 + 128*64 + 128*64 = 65536).
+// 200 for the softmax warpgroups, 48 for the epilogue warpgroup and 64 for the
+// MMA / TMA / allocator warps (2*128*200 + 128*48 + 128*64 = 65536).
 //
 // Every mbarrier wait is bounded (WAIT_LIMIT_NS); on expiry the waiting role records
 // ATTN_ERR_TIMEOUT in the device status word and flags the CTA; every role then
@@ -64,13 +64,6 @@ constexpr uint32_t TMEM_O = 256;        // + D * tile
 // well inside fp16/bf16 range, and O and l stay consistent because both accumulate
 // relative to the same (stale) max, so O / l is unchanged.
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;
-// 2^f on f in [-1/2, 1/2]: degree-3 polynomial with minimax relative error, fitted
-// by the Remez exchange in fit_exp2_poly.py (max relative error 7.5e-5 in fp32
-// evaluation, below the half-ulp of fp16 / bf16 the probabilities are rounded to).
-constexpr float EXP2_C0 = 0.9999280571937561f;
-constexpr float EXP2_C1 = 0.6932609677314758f;
-constexpr float EXP2_C2 = 0.2426111251115799f;
-constexpr float EXP2_C3 = 0.0551716685295105f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s per wait
 constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;   // 0.5 s per drain wait
 
@@ -172,102 +165,71 @@ __device__ __forceinline__ int kv_tiles_for(int q0, int t, int Sq, int Sk) {
 }
 
 // --------------------------------------------------------------------------- softmax
-// 2^x on the FMA pipe (x <= 2^7): n = round(x) by the 1.5*2^23 addition trick,
-// f = x - n, 2^f from the fitted polynomial, and n added to the exponent field.
-// Arguments below -125 are clamped (the result stays a normal number).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;
-    const float f = x - (t - 12582912.f);
-    const float q = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, EXP2_C0);
-    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-
-// Row extreme of 64 raw scores, folded into eight running accumulators: max for a
-// positive scale, min for a negative one (the extreme of scale * s).
-template <bool POS>
-__device__ __forceinline__ void extreme64(const uint32_t* s, float (&a)[8]) {
+// Row max of 64 scores, folded into eight running accumulators.
+__device__ __forceinline__ void max64(const uint32_t* s, float (&a)[8]) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
 #pragma unroll
-        for (int k = 0; k < 8; k += 2) {
-            const float x = __uint_as_float(s[i + 8 * k]);
-            const float y = __uint_as_float(s[i + 8 * k + 8]);
-            a[i] = POS ? ptx::max3(a[i], x, y) : ptx::min3(a[i], x, y);
-        }
+        for (int k = 0; k < 8; k += 2)
+            a[i] = ptx::max3(a[i], __uint_as_float(s[i + 8 * k]), __uint_as_float(s[i + 8 * k + 8]));
     }
 }
 
-template <bool POS>
-__device__ __forceinline__ float extreme128(uint32_t tS, uint32_t (&s)[128]) {
-    float a[8];
+// With a negative scale the scores are negated as they are read (scale * s =
+// |scale| * (-s)), so the softmax below always takes a max and multiplies by |scale|.
+__device__ __forceinline__ void negate32(uint32_t* s, bool negate) {
+    if (negate) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = POS ? -INFINITY : INFINITY;
-    // first half already loaded; the second half's load runs under the first's reduction
-    ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-    ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-    extreme64<POS>(&s[0], a);
-    ptx::tmem_wait_ld();
-    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-    extreme64<POS>(&s[64], a);
-    const float b0 = POS ? ptx::max3(a[0], a[1], a[2]) : ptx::min3(a[0], a[1], a[2]);
-    const float b1 = POS ? ptx::max3(a[3], a[4], a[5]) : ptx::min3(a[3], a[4], a[5]);
-    return POS ? ptx::max3(b0, b1, fmaxf(a[6], a[7])) : ptx::min3(b0, b1, fminf(a[6], a[7]));
+        for (int k = 0; k < 32; ++k) s[k] ^= 0x80000000u;
+    }
 }
 
 // One KV tile of the query row this thread owns: read S_j from TMEM, mask, update the
 // running max (lazily), exponentiate, accumulate the normaliser and write P_j (16-bit)
-// over S_j.  Every POLY-th column pair takes the polynomial 2^x on the FMA pipe, the
-// rest the SFU's ex2 (0 = SFU only).  Returns alpha, the factor O must be scaled by
-// before P_j V_j is added (1 = none).
-template <bool IS_BF16, bool CAUSAL, int POLY>
+// over S_j.  The exponentials run on the SFU (ex2.approx); the scale-and-shift and the
+// row sum use packed f32x2 arithmetic, two columns per instruction.  c = |scale| *
+// log2(e), negate = scale < 0.  Returns alpha, the factor O must be scaled by before
+// P_j V_j is added (1 = none).
+template <bool IS_BF16, bool CAUSAL>
 __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int qrow,
-                                              int q0t, float c_l2, float& m_used, float& l) {
+                                              int q0t, float c, bool negate, float& m_used,
+                                              float& l) {
     uint32_t s[128];
     ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
     ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
     ptx::tmem_wait_ld();
     ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
     ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    // the second half's load runs under the first half's reduction
+    ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+    ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+    negate32(&s[0], negate);
+    negate32(&s[32], negate);
 
     // Keys past `lim` (tile-relative) are invisible: past Sk, or (causal) past qrow.
     const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > q0t);
     int lim = Sk - 1 - kv0;
     if (CAUSAL) lim = min(lim, qrow - kv0);
-    const bool pos = c_l2 >= 0.f;
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = -INFINITY;
+    if (!need_mask) max64(&s[0], a);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+    negate32(&s[64], negate);
+    negate32(&s[96], negate);
     if (need_mask) {
-        // the second half is read here too, so the masking sees all 128 columns
-        ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-        ptx::tmem_wait_ld();
-        ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-        const uint32_t neutral = __float_as_uint(pos ? -INFINITY : INFINITY);
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-            if (c > lim) s[c] = neutral;
+        for (int k = 0; k < 128; ++k)
+            if (k > lim) s[k] = __float_as_uint(-INFINITY);
+        max64(&s[0], a);
     }
-    float mt;
-    if (need_mask) {
-        float a[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = pos ? -INFINITY : INFINITY;
-        if (pos) {
-            extreme64<true>(&s[0], a);
-            extreme64<true>(&s[64], a);
-        } else {
-            extreme64<false>(&s[0], a);
-            extreme64<false>(&s[64], a);
-        }
-#pragma unroll
-        for (int i = 1; i < 8; ++i) a[0] = pos ? fmaxf(a[0], a[i]) : fminf(a[0], a[i]);
-        mt = a[0];
-    } else {
-        mt = pos ? extreme128<true>(tS, s) : extreme128<false>(tS, s);
-    }
-    // every processed tile has a visible key in every row, so mt is finite here
-    const float m_tile = mt * c_l2;
+    max64(&s[64], a);
+    const float mx =
+        ptx::max3(ptx::max3(a[0], a[1], a[2]), ptx::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+    // every processed tile has a visible key in every row, so mx is finite here
+    const float m_tile = mx * c;
     float alpha = 1.f;
     if (j == 0) {
         m_used = m_tile;
@@ -277,40 +239,32 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     }
     const float neg_m = -m_used;
 
-    // p = 2^(s * c - m): scale and shift in one fma
-    float sum0 = 0.f, sum1 = 0.f;
+    // p = 2^(s * c - m): scale and shift in one packed fma per column pair; the row
+    // sum accumulates in a packed pair too
+    const uint64_t c2 = ptx::f32x2(c, c), m2 = ptx::f32x2(neg_m, neg_m);
+    uint64_t acc = ptx::f32x2(0.f, 0.f);
     uint32_t pk[64];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
-        const float x0 = fmaf(__uint_as_float(s[2 * c]), c_l2, neg_m);
-        const float x1 = fmaf(__uint_as_float(s[2 * c + 1]), c_l2, neg_m);
-        float p0, p1;
-        if (POLY > 0 && (c % POLY) == POLY - 1) {
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
-        } else {
-            p0 = ptx::ex2(x0);
-            p1 = ptx::ex2(x1);
-        }
+    for (int k = 0; k < 64; ++k) {
+        float x0, x1;
+        ptx::f32x2_split(
+            ptx::fma2(ptx::f32x2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2, m2),
+            x0, x1);
+        float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
         if (need_mask) {
-            p0 = (2 * c > lim) ? 0.f : p0;
-            p1 = (2 * c + 1 > lim) ? 0.f : p1;
+            p0 = (2 * k > lim) ? 0.f : p0;
+            p1 = (2 * k + 1 > lim) ? 0.f : p1;
         }
-        sum0 += p0;
-        sum1 += p1;
-        pk[c] = pack2<IS_BF16>(p0, p1);
+        acc = ptx::add2(acc, ptx::f32x2(p0, p1));
+        pk[k] = pack2<IS_BF16>(p0, p1);
     }
+    float sum0, sum1;
+    ptx::f32x2_split(acc, sum0, sum1);
     l = l * alpha + (sum0 + sum1);
     ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
     ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
     return alpha;
 }
-
-// Exponent split between the SFU and the FMA pipe: every kPolyEvery-th column pair
-// takes the polynomial.  (On B200 the split changes the time by a few percent either
-// way; it also keeps the softmax within its 192 registers.)
-template <int D>
-constexpr int kPolyEvery = (D == 64) ? 2 : 4;
 
 template <int D, int NS, bool IS_BF16, bool CAUSAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -394,7 +348,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp < 8) {
         // ================================================================ softmax
-        ptx::setmaxnreg_inc<192>();
+        ptx::setmaxnreg_inc<200>();
         const int t = warp >> 2;                    // query tile
         const int wq = warp & 3;                    // TMEM lane quarter
         const int row = wq * 32 + lane;
@@ -404,14 +358,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_base + TMEM_S + 128u * t;
         const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
-        const float c_l2 = p.scale_log2;
+        const float c_abs = fabsf(p.scale_log2);
+        const bool negate = p.scale_log2 < 0.f;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_t; ++j) {
             if (!(ok = warp_wait(ctx, B_SF(t), j & 1))) break;
             ptx::tc_fence_after();
-            const float alpha = softmax_tile<IS_BF16, CAUSAL, kPolyEvery<D>>(
-                tS, j, j * BN, p.Sk, qrow, q0t, c_l2, m_used, l);
+            const float alpha = softmax_tile<IS_BF16, CAUSAL>(
+                tS, j, j * BN, p.Sk, qrow, q0t, c_abs, negate, m_used, l);
             // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
             // bring it to the new max before PV_t,j adds to it
             if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -440,7 +395,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
     } else if (warp < 12) {
         // ================================================================ epilogue
-        ptx::setmaxnreg_dec<64>();
+        ptx::setmaxnreg_dec<48>();
         const int wq = warp & 3;
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
