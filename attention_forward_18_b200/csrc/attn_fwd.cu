@@ -113,10 +113,10 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
 }
 
-template <int D, int NS, bool BF16, bool CAUSAL>
+template <int D, int NS, bool BF16, bool CAUSAL, bool NEG>
 int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const attn::Params& p, int grid, cudaStream_t stream) {
-    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL>;
+    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG>;
     constexpr int smem = attn::SmemLayout<D, NS>::ALLOC;
     static bool attr_set[kMaxDevices];
     static std::mutex mu;
@@ -141,11 +141,17 @@ int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 template <int D>
 constexpr int kStages = (D == 64) ? 5 : 2;
 
+// Negative scales run their own instantiation (scores negated as they are read), so
+// the common case carries no per-element sign handling.
 template <int D, bool BF16>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const attn::Params& p, int grid, bool causal, cudaStream_t s) {
-    if (causal) return launch_one<D, kStages<D>, BF16, true>(tq, tk, tv, p, grid, s);
-    return launch_one<D, kStages<D>, BF16, false>(tq, tk, tv, p, grid, s);
+    const bool neg = p.scale_log2 < 0.f;
+    if (causal)
+        return neg ? launch_one<D, kStages<D>, BF16, true, true>(tq, tk, tv, p, grid, s)
+                   : launch_one<D, kStages<D>, BF16, true, false>(tq, tk, tv, p, grid, s);
+    return neg ? launch_one<D, kStages<D>, BF16, false, true>(tq, tk, tv, p, grid, s)
+               : launch_one<D, kStages<D>, BF16, false, false>(tq, tk, tv, p, grid, s);
 }
 
 int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
@@ -169,6 +175,10 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     p.BH = BH;
     p.n_qp = (Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
+    // A zero scale gives uniform weights over the visible keys; the kernel needs a
+    // nonzero multiplier to keep masked scores at -inf (not -inf * 0 = NaN), and with
+    // 1e-30 every visible weight is 2^(~1e-28) = 1.0f exactly.
+    if (p.scale_log2 == 0.f) p.scale_log2 = 1e-30f;
     p.flags = flags;
     const int grid = p.n_qp * BH;
     const bool c = causal != 0;

@@ -177,53 +177,53 @@ __device__ __forceinline__ void max64(const uint32_t* s, float (&a)[8]) {
 
 // With a negative scale the scores are negated as they are read (scale * s =
 // |scale| * (-s)), so the softmax below always takes a max and multiplies by |scale|.
-__device__ __forceinline__ void negate32(uint32_t* s, bool negate) {
-    if (negate) {
+template <bool NEG>
+__device__ __forceinline__ void load_scores(uint32_t tS, uint32_t (&s)[128], int half) {
+    ptx::tmem_ld32(tS + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&s[64 * half]));
+    ptx::tmem_ld32(tS + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[64 * half + 32]));
+}
+template <bool NEG>
+__device__ __forceinline__ void scores_ready(uint32_t (&s)[128], int half) {
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64 * half]));
+    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64 * half + 32]));
+    if constexpr (NEG) {
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s[k] ^= 0x80000000u;
+        for (int k = 0; k < 64; ++k) s[64 * half + k] ^= 0x80000000u;
     }
 }
 
-// One KV tile of the query row this thread owns: read S_j from TMEM, mask, update the
-// running max (lazily), exponentiate, accumulate the normaliser and write P_j (16-bit)
-// over S_j.  The exponentials run on the SFU (ex2.approx); the scale-and-shift and the
-// row sum use packed f32x2 arithmetic, two columns per instruction.  c = |scale| *
-// log2(e), negate = scale < 0.  Returns alpha, the factor O must be scaled by before
-// P_j V_j is added (1 = none).
-template <bool IS_BF16, bool CAUSAL>
-__device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int qrow,
-                                              int q0t, float c, bool negate, float& m_used,
-                                              float& l) {
+// One KV tile of the query row this thread owns, with the masking decided at compile
+// time (MASK: keys past tile-relative index `lim` are invisible): read S_j from TMEM,
+// update the running max (lazily), exponentiate, accumulate the normaliser and write
+// P_j (16-bit) over S_j.  The exponentials run on the SFU (ex2.approx); the
+// scale-and-shift and the row sum use packed f32x2 arithmetic, two columns per
+// instruction.  c = |scale| * log2(e) > 0 (the host passes 1e-30 for a zero scale:
+// every visible p is then 2^(~1e-28) = 1.0f exactly, the uniform weights a zero
+// scale gives, and masked scores stay -inf).  Returns alpha, the factor O must be
+// scaled by before P_j V_j is added (1 = none).
+template <bool IS_BF16, bool NEG, bool MASK>
+__device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, float c,
+                                                   float& m_used, float& l) {
     uint32_t s[128];
-    ptx::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-    ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    load_scores<NEG>(tS, s, 0);
     ptx::tmem_wait_ld();
-    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+    scores_ready<NEG>(s, 0);
     // the second half's load runs under the first half's reduction
-    ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-    ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-    negate32(&s[0], negate);
-    negate32(&s[32], negate);
-
-    // Keys past `lim` (tile-relative) are invisible: past Sk, or (causal) past qrow.
-    const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > q0t);
-    int lim = Sk - 1 - kv0;
-    if (CAUSAL) lim = min(lim, qrow - kv0);
+    load_scores<NEG>(tS, s, 1);
     float a[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) a[i] = -INFINITY;
-    if (!need_mask) max64(&s[0], a);
-    ptx::tmem_wait_ld();
-    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-    ptx::reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-    negate32(&s[64], negate);
-    negate32(&s[96], negate);
-    if (need_mask) {
+    if constexpr (MASK) {
+        ptx::tmem_wait_ld();
+        scores_ready<NEG>(s, 1);
 #pragma unroll
         for (int k = 0; k < 128; ++k)
             if (k > lim) s[k] = __float_as_uint(-INFINITY);
         max64(&s[0], a);
+    } else {
+        max64(&s[0], a);
+        ptx::tmem_wait_ld();
+        scores_ready<NEG>(s, 1);
     }
     max64(&s[64], a);
     const float mx =
@@ -250,11 +250,8 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
         ptx::f32x2_split(
             ptx::fma2(ptx::f32x2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2, m2),
             x0, x1);
-        float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
-        if (need_mask) {
-            p0 = (2 * k > lim) ? 0.f : p0;
-            p1 = (2 * k + 1 > lim) ? 0.f : p1;
-        }
+        // masked scores are -inf and c > 0, so their p is exactly 0
+        const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
         acc = ptx::add2(acc, ptx::f32x2(p0, p1));
         pk[k] = pack2<IS_BF16>(p0, p1);
     }
@@ -266,7 +263,21 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     return alpha;
 }
 
-template <int D, int NS, bool IS_BF16, bool CAUSAL>
+// The tile's masking is decided once, by a warp-uniform branch, so the unmasked tiles
+// (all but the last and, causally, the diagonal one) run the loops without it.
+template <bool IS_BF16, bool CAUSAL, bool NEG>
+__device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int qrow,
+                                              int q0t, float c, float& m_used, float& l) {
+    const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > q0t);
+    if (need_mask) {
+        int lim = Sk - 1 - kv0;
+        if (CAUSAL) lim = min(lim, qrow - kv0);
+        return softmax_tile_body<IS_BF16, NEG, true>(tS, j, lim, c, m_used, l);
+    }
+    return softmax_tile_body<IS_BF16, NEG, false>(tS, j, 0, c, m_used, l);
+}
+
+template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -359,14 +370,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t tS = tmem + lane_base + TMEM_S + 128u * t;
         const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
         const float c_abs = fabsf(p.scale_log2);
-        const bool negate = p.scale_log2 < 0.f;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_t; ++j) {
             if (!(ok = warp_wait(ctx, B_SF(t), j & 1))) break;
             ptx::tc_fence_after();
-            const float alpha = softmax_tile<IS_BF16, CAUSAL>(
-                tS, j, j * BN, p.Sk, qrow, q0t, c_abs, negate, m_used, l);
+            const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG>(
+                tS, j, j * BN, p.Sk, qrow, q0t, c_abs, m_used, l);
             // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
             // bring it to the new max before PV_t,j adds to it
             if (__any_sync(0xffffffffu, alpha != 1.f)) {
