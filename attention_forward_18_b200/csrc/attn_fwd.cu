@@ -59,9 +59,11 @@ bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool
     return r == CUDA_SUCCESS;
 }
 
-// Per-device facts checked once: compute capability 10.x.
-int check_device() {
+// Per-device facts checked once: compute capability 10.x and the SM count (the
+// persistent grid has one CTA per SM).
+int check_device(int* num_sms) {
     static int verdict[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+    static int sms[kMaxDevices];
     static std::mutex mu;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -70,13 +72,16 @@ int check_device() {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (verdict[dev] == 0) {
-        int major = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        int major = 0, count = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_DEVICE;
         }
-        verdict[dev] = (major == 10) ? 1 : -1;
+        verdict[dev] = (major == 10 && count > 0) ? 1 : -1;
+        sms[dev] = count;
     }
+    if (num_sms) *num_sms = sms[dev];
     return verdict[dev] == 1 ? ATTN_OK : ATTN_ERR_DEVICE;
 }
 
@@ -158,7 +163,8 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
         int Sk, int D, int causal, float scale, int dtype, cudaStream_t stream, unsigned flags) {
     int rc = validate(q, k, v, o, lse, B, H, Sq, Sk, D, scale, dtype);
     if (rc != ATTN_OK) return rc;
-    if ((rc = check_device()) != ATTN_OK) return rc;
+    int num_sms = 0;
+    if ((rc = check_device(&num_sms)) != ATTN_OK) return rc;
 
     const int BH = B * H;
     const bool bf16 = dtype == ATTN_BF16;
@@ -180,7 +186,9 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     // 1e-30 every visible weight is 2^(~1e-28) = 1.0f exactly.
     if (p.scale_log2 == 0.f) p.scale_log2 = 1e-30f;
     p.flags = flags;
-    const int grid = p.n_qp * BH;
+    // persistent: one CTA per SM (at most one per work unit), each walking its units
+    const int n_units = p.n_qp * BH;
+    const int grid = n_units < num_sms ? n_units : num_sms;
     const bool c = causal != 0;
     if (D == 64) return bf16 ? launch_d<64, true>(tq, tk, tv, p, grid, c, stream)
                              : launch_d<64, false>(tq, tk, tv, p, grid, c, stream);
@@ -212,7 +220,7 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
     if (!q_host || !k_host || !v_host || !o_host) return ATTN_ERR_NULLPTR;
     int rc = validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Sq, Sk, D, scale, dtype);
     if (rc != ATTN_OK) return rc;
-    if ((rc = check_device()) != ATTN_OK) return rc;
+    if ((rc = check_device(nullptr)) != ATTN_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t bh = static_cast<size_t>(B) * H;
     const size_t nq = bh * Sq * D * 2, nk = bh * Sk * D * 2;

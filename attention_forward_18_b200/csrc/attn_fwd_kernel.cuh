@@ -83,7 +83,7 @@ struct Params {
 
 template <int D, int NS>
 struct SmemLayout {
-    static_assert(D % CHUNK_ELEMS == 0, "head dim must be a multiple of 64");
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
     static constexpr int NCH = D / CHUNK_ELEMS;
     static constexpr int TILE_BYTES = NCH * CHUNK_BYTES;  // 128 rows x D x 2 bytes
     static constexpr int Q_OFF = 0;                        // two query tiles
@@ -93,8 +93,8 @@ struct SmemLayout {
     static constexpr int FL_OFF = FM_OFF + 2 * BM * 4;      // final sum  float [2][128]
     static constexpr int BAR_OFF = FL_OFF + 2 * BM * 4;
     // q_full[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-    // p_full[2], o_final[2], stats[2], drain
-    static constexpr int NBAR = 2 + 4 * NS + 2 * 4 + 1;
+    // p_full[2], o_final[2], stats[2], o_free[2], q_empty, drain
+    static constexpr int NBAR = 2 + 4 * NS + 2 * 5 + 2;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, error flag
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1024
@@ -277,6 +277,30 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     return softmax_tile_body<IS_BF16, NEG, false>(tS, j, 0, c, m_used, l);
 }
 
+// Work units: (query pair qp, head bh).  Causal grids order them heaviest first (the
+// last query pairs of every head first); non-causal ones keep a head's pairs adjacent
+// so concurrently running units share that head's K/V in L2.
+template <bool CAUSAL>
+__device__ __forceinline__ void unit_coords(int u, int n_qp, int BH, int& qp, int& bh) {
+    if constexpr (CAUSAL) {
+        qp = n_qp - 1 - u / BH;
+        bh = u % BH;
+    } else {
+        qp = u % n_qp;
+        bh = u / n_qp;
+    }
+}
+
+// The r-th unit of this CTA in a boustrophedon order over the grid (round r takes
+// units r*G .. r*G+G-1, in reverse CTA order on odd rounds), so with heaviest-first
+// units every CTA's total stays close to the others'.  -1 when none is left.
+__device__ __forceinline__ int unit_of(int r, int n_units) {
+    const int G = static_cast<int>(gridDim.x);
+    const int b = static_cast<int>(blockIdx.x);
+    const int u = r * G + ((r & 1) ? G - 1 - b : b);
+    return u < n_units ? u : -1;
+}
+
 template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -297,7 +321,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float* s_fm = reinterpret_cast<float*>(smem + L::FM_OFF);
     float* s_fl = reinterpret_cast<float*>(smem + L::FL_OFF);
     const uint32_t bars = sbase + L::BAR_OFF;
-    auto B_QF = [&](int t) { return bars + 8u * t; };
+    auto B_QF = [&](int t) { return bars + 8u * t; };                  // Q_t loaded
     auto B_KF = [&](int s) { return bars + 8u * (2 + s); };
     auto B_KE = [&](int s) { return bars + 8u * (2 + NS + s); };
     auto B_VF = [&](int s) { return bars + 8u * (2 + 2 * NS + s); };
@@ -306,25 +330,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto B_PF = [&](int t) { return bars + 8u * (4 + 4 * NS + t); };   // P_t,j (+ O_t) ready
     auto B_OF = [&](int t) { return bars + 8u * (6 + 4 * NS + t); };   // last PV_t done
     auto B_ST = [&](int t) { return bars + 8u * (8 + 4 * NS + t); };   // final m, l in smem
-    const uint32_t B_DR = bars + 8u * (10 + 4 * NS);
+    auto B_OE = [&](int t) { return bars + 8u * (10 + 4 * NS + t); };  // O_t, m, l read out
+    const uint32_t B_QE = bars + 8u * (12 + 4 * NS);                   // Q tiles free
+    const uint32_t B_DR = bars + 8u * (13 + 4 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     Ctx ctx{reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4)};
+    const int n_units = p.n_qp * p.BH;
 
-    // ---- which rows: causal grids go heaviest query block first
-    int qp, bh;
-    if constexpr (CAUSAL) {
-        qp = p.n_qp - 1 - static_cast<int>(blockIdx.x) / p.BH;
-        bh = static_cast<int>(blockIdx.x) % p.BH;
-    } else {
-        qp = static_cast<int>(blockIdx.x) % p.n_qp;
-        bh = static_cast<int>(blockIdx.x) / p.n_qp;
-    }
-    const int q0 = qp * ROWS_PER_CTA;
-    const int n_t0 = kv_tiles_for<CAUSAL>(q0, 0, p.Sq, p.Sk);
-    const int n_t1 = kv_tiles_for<CAUSAL>(q0, 1, p.Sq, p.Sk);
-    const int n_max = max(n_t0, n_t1);
-
-    // ---- set-up
+    // ---- set-up (once per CTA)
     if (threadIdx.x == 0) {
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(B_QF(t), 1);
@@ -332,6 +345,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_init(B_PF(t), 4);  // one arrival per softmax warp
             ptx::mbar_init(B_OF(t), 1);
             ptx::mbar_init(B_ST(t), 4);  // one arrival per softmax warp
+            ptx::mbar_init(B_OE(t), 4);  // one arrival per epilogue warp
         }
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(B_KF(s), 1);
@@ -339,6 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_init(B_VF(s), 1);
             ptx::mbar_init(B_VE(s), 1);
         }
+        ptx::mbar_init(B_QE, 1);
         ptx::mbar_init(B_DR, 1);
         *ctx.err = 0;
         ptx::fence_mbar_init();
@@ -357,51 +372,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // Barrier phases run on across units: every role visits the same units in the same
+    // order and counts (a) KV tiles per query tile for S / P, (b) KV tiles of the unit
+    // for the K / V ring, (c) units with rows in query tile t for the per-unit
+    // hand-offs (Q, final O, statistics, O read-out).
+
     if (warp < 8) {
         // ================================================================ softmax
         ptx::setmaxnreg_inc<200>();
         const int t = warp >> 2;                    // query tile
         const int wq = warp & 3;                    // TMEM lane quarter
         const int row = wq * 32 + lane;
-        const int q0t = q0 + BM * t;
-        const int qrow = q0t + row;
-        const int n_t = t == 0 ? n_t0 : n_t1;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_base + TMEM_S + 128u * t;
         const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
         const float c_abs = fabsf(p.scale_log2);
-        float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_t; ++j) {
-            if (!(ok = warp_wait(ctx, B_SF(t), j & 1))) break;
-            ptx::tc_fence_after();
-            const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG>(
-                tS, j, j * BN, p.Sk, qrow, q0t, c_abs, m_used, l);
-            // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
-            // bring it to the new max before PV_t,j adds to it
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        uint32_t it = 0;  // KV tiles of this query tile so far (S / P phases)
+        uint32_t ut = 0;  // units with rows in this query tile so far
+        for (int r = 0; ok; ++r) {
+            const int u = unit_of(r, n_units);
+            if (u < 0) break;
+            int qp, bh;
+            unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
+            const int q0t = qp * ROWS_PER_CTA + BM * t;
+            const int qrow = q0t + row;
+            const int n_t = kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, t, p.Sq, p.Sk);
+            float m_used = -INFINITY, l = 0.f;
+            for (int j = 0; j < n_t; ++j, ++it) {
+                if (!(ok = warp_wait(ctx, B_SF(t), it & 1))) break;
+                ptx::tc_fence_after();
+                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG>(
+                    tS, j, j * BN, p.Sk, qrow, q0t, c_abs, m_used, l);
+                // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
+                // bring it to the new max before PV_t,j adds to it
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t ov[32];
-                    ptx::tmem_ld32(tO + 32 * c, ov);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence32(ov);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ov[32];
+                        ptx::tmem_ld32(tO + 32 * c, ov);
+                        ptx::tmem_wait_ld();
+                        ptx::reg_fence32(ov);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-                    ptx::tmem_st32(tO + 32 * c, ov);
+                        for (int e = 0; e < 32; ++e)
+                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        ptx::tmem_st32(tO + 32 * c, ov);
+                    }
                 }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(B_PF(t));
             }
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(B_PF(t));
-        }
-        if (ok && n_t > 0) {
+            if (!ok || n_t == 0) continue;
+            // the epilogue must be done with the previous unit's statistics
+            if (!(ok = warp_wait(ctx, B_OE(t), (ut & 1) ^ 1))) break;
             s_fm[t * BM + row] = m_used;
             s_fl[t * BM + row] = l;
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(B_ST(t));
+            ++ut;
         }
     } else if (warp < 12) {
         // ================================================================ epilogue
@@ -410,43 +440,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int row = wq * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         bool ok = true;
-        // O / l in fp32, one rounding to 16 bits; LSE in natural log
-        for (int t = 0; ok && t < 2; ++t) {
-            const int n_t = t == 0 ? n_t0 : n_t1;
-            if (n_t == 0) continue;
-            if (!(ok = warp_wait(ctx, B_ST(t), 0))) break;
-            if (!(ok = warp_wait(ctx, B_OF(t), 0))) break;
-            ptx::tc_fence_after();
-            const float m_used = s_fm[t * BM + row];
-            const float l = s_fl[t * BM + row];
-            const float inv_l = 1.f / l;
-            const int qrow = q0 + BM * t + row;
-            const bool store = qrow < p.Sq;
-            uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
-                             (static_cast<int64_t>(bh) * p.Sq + qrow) * D;
-            const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
+        uint32_t ut[2] = {0, 0};
+        for (int r = 0; ok; ++r) {
+            const int u = unit_of(r, n_units);
+            if (u < 0) break;
+            int qp, bh;
+            unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
+            // O / l in fp32, one rounding to 16 bits; LSE in natural log
+            for (int t = 0; ok && t < 2; ++t) {
+                if (kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, t, p.Sq, p.Sk) == 0) continue;
+                if (!(ok = warp_wait(ctx, B_ST(t), ut[t] & 1))) break;
+                if (!(ok = warp_wait(ctx, B_OF(t), ut[t] & 1))) break;
+                ptx::tc_fence_after();
+                const float m_used = s_fm[t * BM + row];
+                const float l = s_fl[t * BM + row];
+                const float inv_l = 1.f / l;
+                const int qrow = qp * ROWS_PER_CTA + BM * t + row;
+                const bool store = qrow < p.Sq;
+                uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
+                                 (static_cast<int64_t>(bh) * p.Sq + qrow) * D;
+                const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t ov[32];
-                ptx::tmem_ld32(tO + 32 * c, ov);
-                ptx::tmem_wait_ld();
-                ptx::reg_fence32(ov);
-                uint32_t packed[16];
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t ov[16];
+                    ptx::tmem_ld16(tO + 16 * c, ov);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence16(ov);
+                    uint32_t packed[8];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    packed[e] = pack2<IS_BF16>(__uint_as_float(ov[2 * e]) * inv_l,
-                                               __uint_as_float(ov[2 * e + 1]) * inv_l);
-                if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
-                                            packed[4 * e + 3]);
+                    for (int e = 0; e < 8; ++e)
+                        packed[e] = pack2<IS_BF16>(__uint_as_float(ov[2 * e]) * inv_l,
+                                                   __uint_as_float(ov[2 * e + 1]) * inv_l);
+                    if (store) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
+                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    }
                 }
+                // O_t and the statistics are read: the next unit may overwrite them
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(B_OE(t));
+                ++ut[t];
+                if (store && p.lse != nullptr)
+                    p.lse[static_cast<int64_t>(bh) * p.Sq + qrow] =
+                        (m_used + log2f(l)) * 0.69314718055994530942f;
             }
-            if (store && p.lse != nullptr)
-                p.lse[static_cast<int64_t>(bh) * p.Sq + qrow] =
-                    (m_used + log2f(l)) * 0.69314718055994530942f;
         }
     } else {
         ptx::setmaxnreg_dec<64>();
@@ -456,7 +495,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 constexpr uint32_t fmt = IS_BF16 ? 1u : 0u;
                 constexpr uint32_t idesc_qk = ptx::idesc_f16(fmt, BM, BN, 0);
                 constexpr uint32_t idesc_pv = ptx::idesc_f16(fmt, BM, D, 1);
-                const int n_t[2] = {n_t0, n_t1};
                 // Descriptors: the high word is common to every operand tile; per MMA only
                 // the start-address field of the low word moves, by a compile-time offset.
                 constexpr uint32_t desc_hi = ptx::smem_desc_hi_sw128(1024);
@@ -464,53 +502,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t dk0 = ptx::smem_desc_lo(sK, 16);
                 const uint32_t dv0 = ptx::smem_desc_lo(sV, CHUNK_BYTES);
                 constexpr uint32_t TILE16 = L::TILE_BYTES >> 4;
-                // S_t,j = Q_t K_j^T  (both operands K-major, 128-byte swizzle)
-                auto issue_s = [&](int t, int j) {
+                // S_t = Q_t K^T for the K tile in ring slot `slot`
+                auto issue_s = [&](int t, int slot) {
                     const uint32_t qd = dq0 + static_cast<uint32_t>(t) * TILE16;
-                    const uint32_t kd = dk0 + static_cast<uint32_t>(j % NS) * TILE16;
+                    const uint32_t kd = dk0 + static_cast<uint32_t>(slot) * TILE16;
                     const uint32_t d_tmem = tmem + TMEM_S + 128u * t;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
-                        ptx::mma_ss2(d_tmem, qd + off, kd + off, desc_hi, idesc_qk,
-                                     kk > 0 ? 1u : 0u);
+                    // K-steps of 16: +32 bytes inside a 128-byte row, +16 KB per 64 columns
+                    ptx::mma_ss_off<0, 0>(d_tmem, qd, kd, desc_hi, idesc_qk, 0u);
+                    ptx::mma_ss_off<2, 2>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
+                    ptx::mma_ss_off<4, 4>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
+                    ptx::mma_ss_off<6, 6>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
+                    if constexpr (D == 128) {
+                        constexpr uint32_t C16 = CHUNK_BYTES >> 4;
+                        ptx::mma_ss_off<C16, C16>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
+                        ptx::mma_ss_off<C16 + 2, C16 + 2>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
+                        ptx::mma_ss_off<C16 + 4, C16 + 4>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
+                        ptx::mma_ss_off<C16 + 6, C16 + 6>(d_tmem, qd, kd, desc_hi, idesc_qk, 1u);
                     }
                     ptx::mma_commit(B_SF(t));
                 };
-                // O_t += P_t,j V_j  (P from TMEM, V MN-major in smem)
-                auto issue_pv = [&](int t, int j) {
-                    const uint32_t vd = dv0 + static_cast<uint32_t>(j % NS) * TILE16;
+                // O_t (+)= P_t V for the V tile in ring slot `slot`
+                auto issue_pv = [&](int t, int slot, bool first) {
+                    const uint32_t vd = dv0 + static_cast<uint32_t>(slot) * TILE16;
                     const uint32_t a_tmem = tmem + TMEM_S + 128u * t;
                     const uint32_t d_tmem = tmem + TMEM_O + D * t;
-#pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        ptx::mma_ts2(d_tmem, a_tmem + kk * 8, vd + ((kk * 2048) >> 4), desc_hi,
-                                     idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    if (j == n_t[t] - 1) ptx::mma_commit(B_OF(t));
+                    // K-steps of 16 keys: 8 TMEM columns of P, 2 KB of V
+                    ptx::mma_ts_off<0, 0>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, first ? 0u : 1u);
+                    ptx::mma_ts_off<8, 128>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                    ptx::mma_ts_off<16, 256>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                    ptx::mma_ts_off<24, 384>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                    ptx::mma_ts_off<32, 512>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                    ptx::mma_ts_off<40, 640>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                    ptx::mma_ts_off<48, 768>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                    ptx::mma_ts_off<56, 896>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
                 };
-                bool ok = wait_bounded(ctx, B_QF(0), 0) && wait_bounded(ctx, B_QF(1), 0) &&
-                          wait_bounded(ctx, B_KF(0), 0);
-                if (ok) {
+                bool ok = true;
+                uint32_t kv = 0;          // K/V ring position of the unit's first tile
+                uint32_t pit[2] = {0, 0};  // P phases per query tile
+                uint32_t ut[2] = {0, 0};   // units with rows per query tile
+                uint32_t nu = 0;           // units so far (Q phases)
+                for (int r = 0; ok; ++r) {
+                    const int u = unit_of(r, n_units);
+                    if (u < 0) break;
+                    int qp, bh;
+                    unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
+                    const int n_t[2] = {kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, 0, p.Sq, p.Sk),
+                                        kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, 1, p.Sq, p.Sk)};
+                    const int n_max = max(n_t[0], n_t[1]);
+                    auto slot = [&](int j) { return static_cast<int>((kv + j) % NS); };
+                    auto phase = [&](int j) { return ((kv + j) / NS) & 1u; };
+                    if (!(ok = wait_bounded(ctx, B_QF(0), nu & 1) &&
+                               wait_bounded(ctx, B_QF(1), nu & 1) &&
+                               wait_bounded(ctx, B_KF(slot(0)), phase(0))))
+                        break;
                     ptx::tc_fence_after();
                     for (int t = 0; t < 2; ++t)
-                        if (n_t[t] > 0) issue_s(t, 0);
-                    ptx::mma_commit(B_KE(0));
-                }
-                for (int j = 0; ok && j < n_max; ++j) {
-                    const bool nxt = j + 1 < n_max;
-                    if (nxt && !(ok = wait_bounded(ctx, B_KF((j + 1) % NS), ((j + 1) / NS) & 1)))
-                        break;
-                    if (!(ok = wait_bounded(ctx, B_VF(j % NS), (j / NS) & 1))) break;
-                    for (int t = 0; t < 2; ++t) {
-                        if (j >= n_t[t]) continue;
-                        if (!(ok = wait_bounded(ctx, B_PF(t), j & 1))) break;
-                        ptx::tc_fence_after();
-                        issue_pv(t, j);
-                        if (j + 1 < n_t[t]) issue_s(t, j + 1);
+                        if (n_t[t] > 0) issue_s(t, slot(0));
+                    ptx::mma_commit(B_KE(slot(0)));
+                    if (n_max == 1) ptx::mma_commit(B_QE);  // the unit's last S is issued
+                    for (int j = 0; ok && j < n_max; ++j) {
+                        const bool nxt = j + 1 < n_max;
+                        if (nxt && !(ok = wait_bounded(ctx, B_KF(slot(j + 1)), phase(j + 1))))
+                            break;
+                        if (!(ok = wait_bounded(ctx, B_VF(slot(j)), phase(j)))) break;
+                        for (int t = 0; t < 2; ++t) {
+                            if (j >= n_t[t]) continue;
+                            if (!(ok = wait_bounded(ctx, B_PF(t), pit[t] & 1))) break;
+                            ++pit[t];
+                            // the first P V of a unit overwrites O_t: the epilogue must
+                            // have read the previous unit's O_t
+                            if (j == 0 && !(ok = wait_bounded(ctx, B_OE(t), (ut[t] & 1) ^ 1)))
+                                break;
+                            ptx::tc_fence_after();
+                            issue_pv(t, slot(j), j == 0);
+                            if (j == n_t[t] - 1) ptx::mma_commit(B_OF(t));
+                            if (j + 1 < n_t[t]) issue_s(t, slot(j + 1));
+                        }
+                        if (!ok) break;
+                        ptx::mma_commit(B_VE(slot(j)));
+                        if (nxt) {
+                            ptx::mma_commit(B_KE(slot(j + 1)));
+                            if (j + 1 == n_max - 1) ptx::mma_commit(B_QE);  // last S issued
+                        }
                     }
-                    if (!ok) break;
-                    ptx::mma_commit(B_VE(j % NS));
-                    if (nxt) ptx::mma_commit(B_KE((j + 1) % NS));
+                    for (int t = 0; t < 2; ++t) ut[t] += n_t[t] > 0 ? 1u : 0u;
+                    kv += static_cast<uint32_t>(n_max);
+                    ++nu;
                 }
                 // Every MMA issued above completes before the CTA frees tensor memory.
                 ptx::mma_commit(B_DR);
@@ -521,40 +598,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // ============================================================ producer
             if (lane == 0) {
                 const bool load_q = !(p.flags & FLAG_SKIP_Q_LOAD);
-                if (load_q) {
-                    for (int t = 0; t < 2; ++t) {
-                        ptx::mbar_arrive_expect_tx(B_QF(t), L::TILE_BYTES);
-                        for (int c = 0; c < L::NCH; ++c)
-                            ptx::tma_load_3d(sQ + t * L::TILE_BYTES + c * CHUNK_BYTES, &tm_q,
-                                             B_QF(t), c * CHUNK_ELEMS, q0 + BM * t, bh);
+                uint32_t kv = 0, nu = 0;
+                int64_t last_k = -1, last_v = -1;  // ring positions of the last K / V issued
+                int64_t last_q = -1;               // unit count at the last Q load
+                bool ok = true;
+                for (int r = 0; ok; ++r) {
+                    const int u = unit_of(r, n_units);
+                    if (u < 0) break;
+                    int qp, bh;
+                    unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
+                    const int q0 = qp * ROWS_PER_CTA;
+                    const int n_max = max(kv_tiles_for<CAUSAL>(q0, 0, p.Sq, p.Sk),
+                                          kv_tiles_for<CAUSAL>(q0, 1, p.Sq, p.Sk));
+                    // Q_0, Q_1 are free once the previous unit's S MMAs completed
+                    if (!(ok = wait_bounded(ctx, B_QE, (nu & 1) ^ 1))) break;
+                    if (load_q) {
+                        for (int t = 0; t < 2; ++t) {
+                            ptx::mbar_arrive_expect_tx(B_QF(t), L::TILE_BYTES);
+                            for (int c = 0; c < L::NCH; ++c)
+                                ptx::tma_load_3d(sQ + t * L::TILE_BYTES + c * CHUNK_BYTES, &tm_q,
+                                                 B_QF(t), c * CHUNK_ELEMS, q0 + BM * t, bh);
+                        }
+                        last_q = nu;
                     }
-                }
-                int last_k = -1, last_v = -1;  // last issued tile index
-                for (int j = 0; j < n_max; ++j) {
-                    const int s = j % NS;
-                    const uint32_t ph = (j / NS) & 1;
-                    if (!wait_bounded(ctx, B_KE(s), ph ^ 1)) break;
-                    ptx::mbar_arrive_expect_tx(B_KF(s), L::TILE_BYTES);
-                    for (int c = 0; c < L::NCH; ++c)
-                        ptx::tma_load_3d(sK + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_k,
-                                         B_KF(s), c * CHUNK_ELEMS, j * BN, bh);
-                    last_k = j;
-                    if (!wait_bounded(ctx, B_VE(s), ph ^ 1)) break;
-                    ptx::mbar_arrive_expect_tx(B_VF(s), L::TILE_BYTES);
-                    for (int c = 0; c < L::NCH; ++c)
-                        ptx::tma_load_3d(sV + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_v,
-                                         B_VF(s), c * CHUNK_ELEMS, j * BN, bh);
-                    last_v = j;
+                    for (int j = 0; ok && j < n_max; ++j) {
+                        const uint32_t pos = kv + j;
+                        const int s = static_cast<int>(pos % NS);
+                        const uint32_t ph = (pos / NS) & 1;
+                        if (!(ok = wait_bounded(ctx, B_KE(s), ph ^ 1))) break;
+                        ptx::mbar_arrive_expect_tx(B_KF(s), L::TILE_BYTES);
+                        for (int c = 0; c < L::NCH; ++c)
+                            ptx::tma_load_3d(sK + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_k,
+                                             B_KF(s), c * CHUNK_ELEMS, j * BN, bh);
+                        last_k = pos;
+                        if (!(ok = wait_bounded(ctx, B_VE(s), ph ^ 1))) break;
+                        ptx::mbar_arrive_expect_tx(B_VF(s), L::TILE_BYTES);
+                        for (int c = 0; c < L::NCH; ++c)
+                            ptx::tma_load_3d(sV + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_v,
+                                             B_VF(s), c * CHUNK_ELEMS, j * BN, bh);
+                        last_v = pos;
+                    }
+                    kv += static_cast<uint32_t>(n_max);
+                    ++nu;
                 }
                 // Let every copy this thread started land before the CTA can exit.
-                if (load_q) {
-                    wait_drain(B_QF(0), 0);
-                    wait_drain(B_QF(1), 0);
+                if (last_q >= 0) {
+                    wait_drain(B_QF(0), static_cast<uint32_t>(last_q) & 1);
+                    wait_drain(B_QF(1), static_cast<uint32_t>(last_q) & 1);
                 }
-                for (int j = (last_k - NS + 1 > 0 ? last_k - NS + 1 : 0); j <= last_k; ++j)
-                    wait_drain(B_KF(j % NS), (j / NS) & 1);
-                for (int j = (last_v - NS + 1 > 0 ? last_v - NS + 1 : 0); j <= last_v; ++j)
-                    wait_drain(B_VF(j % NS), (j / NS) & 1);
+                for (int64_t q = (last_k - NS + 1 > 0 ? last_k - NS + 1 : 0); q <= last_k; ++q)
+                    wait_drain(B_KF(static_cast<int>(q % NS)), (q / NS) & 1);
+                for (int64_t q = (last_v - NS + 1 > 0 ? last_v - NS + 1 : 0); q <= last_v; ++q)
+                    wait_drain(B_VF(static_cast<int>(q % NS)), (q / NS) & 1);
             }
             __syncwarp();
         }
