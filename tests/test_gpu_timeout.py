@@ -1,0 +1,52 @@
+"""Failure detection without a GPU fault: a pipeline wait that nothing will satisfy
+must end with ATTN_ERR_TIMEOUT in the device status word after its bounded limit,
+and the context must stay usable.
+
+The test-only flag of attn_fwd_debug makes the TMA producer skip the Q loads, so
+the MMA thread's first wait (for Q) is on a barrier nothing will complete: it gives
+up after its 2 s limit, flags the CTA, and every role leaves its loop, drains its own
+copies / MMAs, and the CTA frees its tensor memory and exits.  No trap, no fault."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import attention_forward_18_b200 as af
+from parity import check_full
+from workloads import make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def test_unsatisfied_wait_reports_timeout_and_context_survives():
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, 256, 256, 64, "f16", 21))
+    o = torch.zeros_like(q)
+    lse = torch.zeros((1, 2, 256), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert af.attn_fwd_status() == 0
+    t0 = time.monotonic()
+    rc = af.attn_fwd_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           lse.data_ptr(), 1, 2, 256, 256, 64, 0, 0.125, af.ATTN_F16, stream, 1)
+    assert rc == af.ATTN_OK                   # the launch itself succeeds
+    status = af.attn_fwd_status()             # synchronises the stream
+    elapsed = time.monotonic() - t0
+    assert status == af.ATTN_ERR_TIMEOUT
+    assert 1.0 < elapsed < 30.0               # the 2 s limit, not a hang
+    assert af.attn_fwd_status() == 0          # reading cleared the word
+    # the context is intact: a normal call still gives the oracle's answer
+    check_full(1, 2, 200, 300, 64, "f16", True, seed=22)
+
+
+def test_debug_entry_without_flags_is_the_normal_pass():
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, 130, 130, 128, "bf16", 23))
+    o1, l1 = af.attention(q, k, v, causal=True)
+    o2 = torch.empty_like(q)
+    l2 = torch.empty_like(l1)
+    rc = af.attn_fwd_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(),
+                           l2.data_ptr(), 1, 2, 130, 130, 128, 1, 1 / np.sqrt(128),
+                           af.ATTN_BF16, torch.cuda.current_stream().cuda_stream, 0)
+    assert rc == af.ATTN_OK
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert af.attn_fwd_status() == 0
