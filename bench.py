@@ -44,8 +44,9 @@ FLUSH_BYTES = 256 << 20
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of
-# the same kernel build (see profiles/); None when no capture matches the build.
-NCU_TRAFFIC_BYTES = {}
+# the same kernel build (profiles/attn_fwd_kernel_D64_f16_B4H16S1024_bench_workload.md);
+# a workload without a matching capture reports null.
+NCU_TRAFFIC_BYTES = {"C2-noncausal": 25224960}
 
 
 def parse():
