@@ -40,9 +40,11 @@ ATTN_ERR_TIMEOUT = -8
 ATTN_ERR_SCALE = -9
 ATTN_ERR_ALIAS = -10
 ATTN_ERR_DEVICE = -11
+ATTN_ERR_WORKSPACE = -12
 
 # Every symbol include/attn_fwd.h declares.
-EXPORTS = ("attn_fwd", "attn_fwd_host", "attn_fwd_status", "attn_fwd_strerror",
+EXPORTS = ("attn_fwd", "attn_fwd_host", "attn_fwd_splitkv", "attn_fwd_splitkv_workspace_bytes",
+           "attn_fwd_splitkv_default_splits", "attn_fwd_status", "attn_fwd_strerror",
            "attn_fwd_abi_version", "attn_fwd_debug")
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -54,6 +56,12 @@ _lib.attn_fwd_debug.argtypes = [_vp] * 5 + _SIZES + [ctypes.c_uint]
 _lib.attn_fwd_debug.restype = _i
 _lib.attn_fwd_host.argtypes = [_vp] * 10 + _SIZES
 _lib.attn_fwd_host.restype = _i
+_lib.attn_fwd_splitkv.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _i, _i, _vp, ctypes.c_size_t, _vp]
+_lib.attn_fwd_splitkv.restype = _i
+_lib.attn_fwd_splitkv_workspace_bytes.argtypes = [_i] * 5
+_lib.attn_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
+_lib.attn_fwd_splitkv_default_splits.argtypes = [_i] * 4
+_lib.attn_fwd_splitkv_default_splits.restype = _i
 _lib.attn_fwd_status.argtypes = [_vp, ctypes.POINTER(_i)]
 _lib.attn_fwd_status.restype = _i
 _lib.attn_fwd_strerror.argtypes = [_i]
@@ -99,6 +107,21 @@ def attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev,
     return _lib.attn_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev,
                               o_dev, lse_dev, B, H, Sq, Sk, D, int(causal), float(scale),
                               int(dtype), stream)
+
+
+def attn_fwd_splitkv(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype, n_splits,
+                     workspace, workspace_bytes, stream):
+    return _lib.attn_fwd_splitkv(q, k, v, o, lse, B, H, Sq, Sk, D, int(causal), float(scale),
+                                 int(dtype), int(n_splits), workspace, int(workspace_bytes),
+                                 stream)
+
+
+def splitkv_workspace_bytes(B, H, Sq, D, n_splits):
+    return _lib.attn_fwd_splitkv_workspace_bytes(B, H, Sq, D, n_splits)
+
+
+def splitkv_default_splits(B, H, Sq, Sk):
+    return _lib.attn_fwd_splitkv_default_splits(B, H, Sq, Sk)
 
 
 def attn_fwd_status(stream=None):
@@ -166,6 +189,33 @@ def attention(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=Tr
     return out, lse
 
 
+def attention_splitkv(q, k, v, causal=False, scale=None, n_splits=None, out=None, lse=None,
+                      with_lse=True, workspace=None, stream=None):
+    """Split-KV pass (decode-shaped inputs): n_splits KV ranges per (query block, head)
+    merged by their log-sum-exp.  The workspace is allocated with torch unless given.
+    Returns (o, lse or None)."""
+    torch = _torch()
+    B, H, Sq, Sk, D = _shape(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if n_splits is None:
+        n_splits = splitkv_default_splits(B, H, Sq, Sk)
+    nbytes = splitkv_workspace_bytes(B, H, Sq, D, n_splits)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    rc = _lib.attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr() if lse is not None else None, B, H, Sq, Sk, D,
+                               int(bool(causal)), float(scale), _dtype_code(q), int(n_splits),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               _stream_ptr(stream))
+    _check(rc, "attn_fwd_splitkv")
+    return out, lse
+
+
 def attention_host(q, k, v, staging, causal=False, scale=None, out=None, lse=None,
                    stream=None):
     """The pass from (pinned) host tensors through attn_fwd_host.  `staging` is a tuple
@@ -188,6 +238,7 @@ def attention_host(q, k, v, staging, causal=False, scale=None, out=None, lse=Non
     return out, lse
 
 
-__all__ = ["attn_fwd", "attn_fwd_host", "attn_fwd_status", "attn_fwd_debug", "attention",
-           "attention_host", "strerror", "abi_version", "AttnError", "ATTN_F16", "ATTN_BF16",
-           "LIB_PATH", "EXPORTS"]
+__all__ = ["attn_fwd", "attn_fwd_host", "attn_fwd_splitkv", "attn_fwd_status", "attn_fwd_debug",
+           "attention", "attention_splitkv", "attention_host", "splitkv_workspace_bytes",
+           "splitkv_default_splits", "strerror", "abi_version", "AttnError", "ATTN_F16",
+           "ATTN_BF16", "LIB_PATH", "EXPORTS"]

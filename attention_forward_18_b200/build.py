@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "attn_fwd.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("attn_fwd_kernel.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("attn_fwd_kernel.cuh", "attn_merge.cuh", "ptx.cuh")] + [
     os.path.join(ROOT, "include", "attn_fwd.h")]
 LIB = os.path.join(HERE, "libattn_fwd.so")
 

@@ -11,12 +11,14 @@
 
 #include "attn_fwd.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_merge.cuh"
 
 namespace {
 
 constexpr int kMaxSeq = 1 << 24;
 constexpr int kMaxHeads = 1 << 24;
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSplits = 1024;
 
 // cuTensorMapEncodeTiled, fetched through the runtime so the library needs no
 // link against libcuda.
@@ -118,10 +120,10 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
 }
 
-template <int D, int NS, bool BF16, bool CAUSAL, bool NEG>
+template <int D, int NS, bool BF16, bool CAUSAL, bool NEG, bool SPLIT>
 int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const attn::Params& p, int grid, cudaStream_t stream) {
-    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG>;
+    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG, SPLIT>;
     constexpr int smem = attn::SmemLayout<D, NS>::ALLOC;
     static bool attr_set[kMaxDevices];
     static std::mutex mu;
@@ -148,21 +150,75 @@ constexpr int kStages = (D == 64) ? 5 : 2;
 
 // Negative scales run their own instantiation (scores negated as they are read), so
 // the common case carries no per-element sign handling.
-template <int D, bool BF16>
+template <int D, bool BF16, bool SPLIT>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const attn::Params& p, int grid, bool causal, cudaStream_t s) {
     const bool neg = p.scale_log2 < 0.f;
+    constexpr int NS = kStages<D>;
     if (causal)
-        return neg ? launch_one<D, kStages<D>, BF16, true, true>(tq, tk, tv, p, grid, s)
-                   : launch_one<D, kStages<D>, BF16, true, false>(tq, tk, tv, p, grid, s);
-    return neg ? launch_one<D, kStages<D>, BF16, false, true>(tq, tk, tv, p, grid, s)
-               : launch_one<D, kStages<D>, BF16, false, false>(tq, tk, tv, p, grid, s);
+        return neg ? launch_one<D, NS, BF16, true, true, SPLIT>(tq, tk, tv, p, grid, s)
+                   : launch_one<D, NS, BF16, true, false, SPLIT>(tq, tk, tv, p, grid, s);
+    return neg ? launch_one<D, NS, BF16, false, true, SPLIT>(tq, tk, tv, p, grid, s)
+               : launch_one<D, NS, BF16, false, false, SPLIT>(tq, tk, tv, p, grid, s);
 }
 
+template <bool SPLIT>
+int launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const attn::Params& p, int grid, int D, bool bf16, bool causal,
+               cudaStream_t s) {
+    if (D == 64) return bf16 ? launch_d<64, true, SPLIT>(tq, tk, tv, p, grid, causal, s)
+                             : launch_d<64, false, SPLIT>(tq, tk, tv, p, grid, causal, s);
+    return bf16 ? launch_d<128, true, SPLIT>(tq, tk, tv, p, grid, causal, s)
+                : launch_d<128, false, SPLIT>(tq, tk, tv, p, grid, causal, s);
+}
+
+// Workspace of a split pass: partial O [n_splits, B*H, Sq, D] fp32, then partial LSE
+// [n_splits, B*H, Sq] fp32 at the next 256-byte boundary.
+size_t ws_o_bytes(int B, int H, int Sq, int D, int n_splits) {
+    const size_t b = static_cast<size_t>(n_splits) * B * H * Sq * D * 4;
+    return (b + 255) & ~static_cast<size_t>(255);
+}
+size_t ws_bytes(int B, int H, int Sq, int D, int n_splits) {
+    return ws_o_bytes(B, H, Sq, D, n_splits) + static_cast<size_t>(n_splits) * B * H * Sq * 4;
+}
+
+int launch_merge(const float* ws_o, const float* ws_lse, void* o, float* lse, int n_splits,
+                 int64_t rows, int D, bool bf16, cudaStream_t s) {
+    const int64_t threads = rows * 32;
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    if (D == 64) {
+        if (bf16) attn::attn_splitkv_merge_kernel<64, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+        else attn::attn_splitkv_merge_kernel<64, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+    } else {
+        if (bf16) attn::attn_splitkv_merge_kernel<128, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+        else attn::attn_splitkv_merge_kernel<128, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+    }
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// n_splits == 0: the whole pass (16-bit O and LSE written by the attention kernel);
+// n_splits >= 1: a split pass through `workspace`, then the merge kernel.
 int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
-        int Sk, int D, int causal, float scale, int dtype, cudaStream_t stream, unsigned flags) {
+        int Sk, int D, int causal, float scale, int dtype, cudaStream_t stream, unsigned flags,
+        int n_splits = 0, void* workspace = nullptr, size_t workspace_bytes = 0) {
     int rc = validate(q, k, v, o, lse, B, H, Sq, Sk, D, scale, dtype);
     if (rc != ATTN_OK) return rc;
+    if (n_splits < 0 || n_splits > kMaxSplits) return ATTN_ERR_SHAPE;
+    if (n_splits > 0) {
+        // the merge kernel runs one warp per (head, query row) in a 1-D grid
+        if (static_cast<int64_t>(B) * H * Sq > static_cast<int64_t>(INT_MAX) * 8)
+            return ATTN_ERR_SHAPE;
+        if (!workspace) return ATTN_ERR_NULLPTR;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_ALIGN;
+        const size_t need = ws_bytes(B, H, Sq, D, n_splits);
+        if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+        const size_t nq = static_cast<size_t>(B) * H * Sq * D * 2;
+        const size_t nk = static_cast<size_t>(B) * H * Sk * D * 2;
+        if (overlaps(workspace, need, q, nq) || overlaps(workspace, need, k, nk) ||
+            overlaps(workspace, need, v, nk) || overlaps(workspace, need, o, nq) ||
+            (lse && overlaps(workspace, need, lse, static_cast<size_t>(B) * H * Sq * 4)))
+            return ATTN_ERR_ALIAS;
+    }
     int num_sms = 0;
     if ((rc = check_device(&num_sms)) != ATTN_OK) return rc;
 
@@ -180,6 +236,13 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     p.Sk = Sk;
     p.BH = BH;
     p.n_qp = (Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    const int n_kv = (Sk + attn::BN - 1) / attn::BN;
+    p.n_splits = n_splits > 0 ? n_splits : 1;
+    p.chunk_tiles = (n_kv + p.n_splits - 1) / p.n_splits;
+    p.ws_o = n_splits > 0 ? static_cast<float*>(workspace) : nullptr;
+    p.ws_lse = n_splits > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                       ws_o_bytes(B, H, Sq, D, n_splits))
+                            : nullptr;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634074);
     // A zero scale gives uniform weights over the visible keys; the kernel needs a
     // nonzero multiplier to keep masked scores at -inf (not -inf * 0 = NaN), and with
@@ -187,13 +250,15 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     if (p.scale_log2 == 0.f) p.scale_log2 = 1e-30f;
     p.flags = flags;
     // persistent: one CTA per SM (at most one per work unit), each walking its units
-    const int n_units = p.n_qp * BH;
-    const int grid = n_units < num_sms ? n_units : num_sms;
+    const int64_t n_units = static_cast<int64_t>(p.n_qp) * BH * p.n_splits;
+    if (n_units > INT_MAX) return ATTN_ERR_SHAPE;
+    const int grid = n_units < num_sms ? static_cast<int>(n_units) : num_sms;
     const bool c = causal != 0;
-    if (D == 64) return bf16 ? launch_d<64, true>(tq, tk, tv, p, grid, c, stream)
-                             : launch_d<64, false>(tq, tk, tv, p, grid, c, stream);
-    return bf16 ? launch_d<128, true>(tq, tk, tv, p, grid, c, stream)
-                : launch_d<128, false>(tq, tk, tv, p, grid, c, stream);
+    if (n_splits == 0) return launch_any<false>(tq, tk, tv, p, grid, D, bf16, c, stream);
+    rc = launch_any<true>(tq, tk, tv, p, grid, D, bf16, c, stream);
+    if (rc != ATTN_OK) return rc;
+    return launch_merge(p.ws_o, p.ws_lse, o, lse, n_splits, static_cast<int64_t>(BH) * Sq, D,
+                        bf16, stream);
 }
 
 }  // namespace
@@ -244,6 +309,36 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
     return ATTN_OK;
 }
 
+size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_splits) {
+    if (B < 1 || H < 1 || Sq < 1 || (D != 64 && D != 128) || n_splits < 1 ||
+        n_splits > kMaxSplits)
+        return 0;
+    return ws_bytes(B, H, Sq, D, n_splits);
+}
+
+int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk) {
+    if (B < 1 || H < 1 || Sq < 1 || Sk < 1) return 0;
+    int num_sms = 0;
+    if (check_device(&num_sms) != ATTN_OK) num_sms = 148;
+    const int64_t units = static_cast<int64_t>((Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA) *
+                          B * H;
+    const int n_kv = (Sk + attn::BN - 1) / attn::BN;
+    // about two units per SM, at least one KV tile per range
+    int64_t s = (2 * static_cast<int64_t>(num_sms) + units - 1) / units;
+    if (s > n_kv) s = n_kv;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return s < 1 ? 1 : static_cast<int>(s);
+}
+
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Sq, int Sk, int D, int causal, float scale, int dtype,
+                     int n_splits, void* workspace, size_t workspace_bytes,
+                     attn_stream_t stream) {
+    if (n_splits < 1) return ATTN_ERR_SHAPE;
+    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+               reinterpret_cast<cudaStream_t>(stream), 0u, n_splits, workspace, workspace_bytes);
+}
+
 int attn_fwd_status(attn_stream_t stream, int* device_status) {
     if (!device_status) return ATTN_ERR_NULLPTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -276,6 +371,7 @@ const char* attn_fwd_strerror(int code) {
         case ATTN_ERR_SCALE: return "scale is not finite";
         case ATTN_ERR_ALIAS: return "output overlaps an input";
         case ATTN_ERR_DEVICE: return "no usable sm_100 CUDA device";
+        case ATTN_ERR_WORKSPACE: return "workspace smaller than attn_fwd_splitkv_workspace_bytes";
         default: return "unknown error code";
     }
 }

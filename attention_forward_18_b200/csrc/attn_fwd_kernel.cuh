@@ -74,9 +74,13 @@ constexpr int STATUS_TIMEOUT = -8;  // ATTN_ERR_TIMEOUT
 constexpr uint32_t FLAG_SKIP_Q_LOAD = 1u;
 
 struct Params {
-    void* o;            // [BH, Sq, D] 16-bit
-    float* lse;         // [BH, Sq] fp32, may be null
+    void* o;            // [BH, Sq, D] 16-bit (whole pass)
+    float* lse;         // [BH, Sq] fp32, may be null (whole pass)
+    float* ws_o;        // split-KV: [n_splits, BH, Sq, D] fp32 partial O (normalised)
+    float* ws_lse;      // split-KV: [n_splits, BH, Sq] fp32 partial LSE
     int Sq, Sk, BH, n_qp;
+    int n_splits;       // KV ranges per (query pair, head); 1 for the whole pass
+    int chunk_tiles;    // KV tiles per range
     float scale_log2;   // scale * log2(e)
     uint32_t flags;
 };
@@ -152,16 +156,40 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     else return ptx::pack_f16x2(lo, hi);
 }
 
-// Number of 128-key tiles query tile `t` of the CTA at row q0 needs (0 when the tile
-// lies past Sq).  Causal: keys up to the tile's last valid row (top-left mask).
+// One work unit: query pair qp (rows qp*256 .. +255) of head bh, over the KV tiles
+// [kv0, kv0 + n[t]) for query tile t (0 tiles when the query tile lies past Sq or,
+// causally, before the range).  Units are numbered so that causal grids go heaviest
+// first (the last query pairs of every head first) and non-causal grids keep a head's
+// query pairs adjacent (concurrent units share its K/V in L2); the KV ranges of one
+// (query pair, head) are adjacent.
+struct Unit {
+    int qp, bh, split, kv0;
+    int n[2];
+};
+
 template <bool CAUSAL>
-__device__ __forceinline__ int kv_tiles_for(int q0, int t, int Sq, int Sk) {
-    const int first = q0 + BM * t;
-    if (first >= Sq) return 0;
-    const int n_all = (Sk + BN - 1) / BN;
-    if (!CAUSAL) return n_all;
-    const int last_row = min(first + BM - 1, Sq - 1);
-    return min(n_all, last_row / BN + 1);
+__device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
+    Unit w;
+    w.split = u % p.n_splits;
+    const int rest = u / p.n_splits;
+    if constexpr (CAUSAL) {
+        w.qp = p.n_qp - 1 - rest / p.BH;
+        w.bh = rest % p.BH;
+    } else {
+        w.qp = rest % p.n_qp;
+        w.bh = rest / p.n_qp;
+    }
+    const int n_all = (p.Sk + BN - 1) / BN;
+    w.kv0 = w.split * p.chunk_tiles;
+    const int kv_end = min(n_all, w.kv0 + p.chunk_tiles);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int first = w.qp * ROWS_PER_CTA + BM * t;
+        int end = kv_end;
+        if (CAUSAL) end = min(end, (min(first + BM - 1, p.Sq - 1)) / BN + 1);
+        w.n[t] = (first >= p.Sq) ? 0 : max(0, end - w.kv0);
+    }
+    return w;
 }
 
 // --------------------------------------------------------------------------- softmax
@@ -237,7 +265,9 @@ __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, 
         alpha = ptx::ex2(m_used - m_tile);
         m_used = m_tile;
     }
-    const float neg_m = -m_used;
+    // a row with no visible key so far (possible in a KV range of a split pass) keeps
+    // m = -inf; its p are 0 and nothing may compute -inf - (-inf)
+    const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
 
     // p = 2^(s * c - m): scale and shift in one packed fma per column pair; the row
     // sum accumulates in a packed pair too
@@ -277,20 +307,6 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     return softmax_tile_body<IS_BF16, NEG, false>(tS, j, 0, c, m_used, l);
 }
 
-// Work units: (query pair qp, head bh).  Causal grids order them heaviest first (the
-// last query pairs of every head first); non-causal ones keep a head's pairs adjacent
-// so concurrently running units share that head's K/V in L2.
-template <bool CAUSAL>
-__device__ __forceinline__ void unit_coords(int u, int n_qp, int BH, int& qp, int& bh) {
-    if constexpr (CAUSAL) {
-        qp = n_qp - 1 - u / BH;
-        bh = u % BH;
-    } else {
-        qp = u % n_qp;
-        bh = u / n_qp;
-    }
-}
-
 // The r-th unit of this CTA in a boustrophedon order over the grid (round r takes
 // units r*G .. r*G+G-1, in reverse CTA order on odd rounds), so with heaviest-first
 // units every CTA's total stays close to the others'.  -1 when none is left.
@@ -301,7 +317,7 @@ __device__ __forceinline__ int unit_of(int r, int n_units) {
     return u < n_units ? u : -1;
 }
 
-template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG>
+template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -335,7 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t B_DR = bars + 8u * (13 + 4 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     Ctx ctx{reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4)};
-    const int n_units = p.n_qp * p.BH;
+    const int n_units = p.n_qp * p.BH * p.n_splits;
 
     // ---- set-up (once per CTA)
     if (threadIdx.x == 0) {
@@ -393,17 +409,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int u = unit_of(r, n_units);
             if (u < 0) break;
-            int qp, bh;
-            unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
-            const int q0t = qp * ROWS_PER_CTA + BM * t;
+            const Unit w = decode_unit<CAUSAL>(u, p);
+            const int q0t = w.qp * ROWS_PER_CTA + BM * t;
             const int qrow = q0t + row;
-            const int n_t = kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, t, p.Sq, p.Sk);
+            const int n_t = w.n[t];
             float m_used = -INFINITY, l = 0.f;
             for (int j = 0; j < n_t; ++j, ++it) {
                 if (!(ok = warp_wait(ctx, B_SF(t), it & 1))) break;
                 ptx::tc_fence_after();
                 const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG>(
-                    tS, j, j * BN, p.Sk, qrow, q0t, c_abs, m_used, l);
+                    tS, j, (w.kv0 + j) * BN, p.Sk, qrow, q0t, c_abs, m_used, l);
                 // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
                 // bring it to the new max before PV_t,j adds to it
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -444,37 +459,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int u = unit_of(r, n_units);
             if (u < 0) break;
-            int qp, bh;
-            unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
-            // O / l in fp32, one rounding to 16 bits; LSE in natural log
+            const Unit w = decode_unit<CAUSAL>(u, p);
+            const int64_t head_row = static_cast<int64_t>(w.split) * p.BH + w.bh;
             for (int t = 0; ok && t < 2; ++t) {
-                if (kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, t, p.Sq, p.Sk) == 0) continue;
+                const int qrow = w.qp * ROWS_PER_CTA + BM * t + row;
+                const bool store = qrow < p.Sq;
+                if (w.n[t] == 0) {
+                    // split pass: no key of this range is visible to these rows
+                    if (SPLIT && store) {
+                        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D);
+#pragma unroll 1
+                        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        p.ws_lse[head_row * p.Sq + qrow] = -INFINITY;
+                    }
+                    continue;
+                }
                 if (!(ok = warp_wait(ctx, B_ST(t), ut[t] & 1))) break;
                 if (!(ok = warp_wait(ctx, B_OF(t), ut[t] & 1))) break;
                 ptx::tc_fence_after();
                 const float m_used = s_fm[t * BM + row];
                 const float l = s_fl[t * BM + row];
-                const float inv_l = 1.f / l;
-                const int qrow = qp * ROWS_PER_CTA + BM * t + row;
-                const bool store = qrow < p.Sq;
-                uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
-                                 (static_cast<int64_t>(bh) * p.Sq + qrow) * D;
+                // l = 0 only for a row with no visible key in a split range
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
+                const float lse_row =
+                    l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
                 const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
+                if constexpr (SPLIT) {
+                    // partial O / l and LSE of this KV range, fp32
+                    float* orow = p.ws_o + (head_row * p.Sq + qrow) * D;
 #pragma unroll 1
-                for (int c = 0; c < D / 16; ++c) {
-                    uint32_t ov[16];
-                    ptx::tmem_ld16(tO + 16 * c, ov);
-                    ptx::tmem_wait_ld();
-                    ptx::reg_fence16(ov);
-                    uint32_t packed[8];
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t ov[16];
+                        ptx::tmem_ld16(tO + 16 * c, ov);
+                        ptx::tmem_wait_ld();
+                        ptx::reg_fence16(ov);
+                        if (store) {
+                            float4* dst = reinterpret_cast<float4*>(orow + 16 * c);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        packed[e] = pack2<IS_BF16>(__uint_as_float(ov[2 * e]) * inv_l,
-                                                   __uint_as_float(ov[2 * e + 1]) * inv_l);
-                    if (store) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
-                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                            for (int e = 0; e < 4; ++e)
+                                dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                                     __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                                     __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                                     __uint_as_float(ov[4 * e + 3]) * inv_l);
+                        }
+                    }
+                } else {
+                    // O / l in fp32, one rounding to 16 bits; LSE in natural log
+                    uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
+                                     (static_cast<int64_t>(w.bh) * p.Sq + qrow) * D;
+#pragma unroll 1
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t ov[16];
+                        ptx::tmem_ld16(tO + 16 * c, ov);
+                        ptx::tmem_wait_ld();
+                        ptx::reg_fence16(ov);
+                        uint32_t packed[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            packed[e] = pack2<IS_BF16>(__uint_as_float(ov[2 * e]) * inv_l,
+                                                       __uint_as_float(ov[2 * e + 1]) * inv_l);
+                        if (store) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + 16 * c);
+                            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                        }
                     }
                 }
                 // O_t and the statistics are read: the next unit may overwrite them
@@ -482,9 +530,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(B_OE(t));
                 ++ut[t];
-                if (store && p.lse != nullptr)
-                    p.lse[static_cast<int64_t>(bh) * p.Sq + qrow] =
-                        (m_used + log2f(l)) * 0.69314718055994530942f;
+                if (store) {
+                    if constexpr (SPLIT)
+                        p.ws_lse[head_row * p.Sq + qrow] = lse_row;
+                    else if (p.lse != nullptr)
+                        p.lse[static_cast<int64_t>(w.bh) * p.Sq + qrow] = lse_row;
+                }
             }
         }
     } else {
@@ -544,11 +595,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
-                    int qp, bh;
-                    unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
-                    const int n_t[2] = {kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, 0, p.Sq, p.Sk),
-                                        kv_tiles_for<CAUSAL>(qp * ROWS_PER_CTA, 1, p.Sq, p.Sk)};
+                    const Unit w = decode_unit<CAUSAL>(u, p);
+                    const int n_t[2] = {w.n[0], w.n[1]};
                     const int n_max = max(n_t[0], n_t[1]);
+                    if (n_max == 0) continue;  // a split range no query row of the unit sees
                     auto slot = [&](int j) { return static_cast<int>((kv + j) % NS); };
                     auto phase = [&](int j) { return ((kv + j) / NS) & 1u; };
                     if (!(ok = wait_bounded(ctx, B_QF(0), nu & 1) &&
@@ -605,11 +655,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
-                    int qp, bh;
-                    unit_coords<CAUSAL>(u, p.n_qp, p.BH, qp, bh);
-                    const int q0 = qp * ROWS_PER_CTA;
-                    const int n_max = max(kv_tiles_for<CAUSAL>(q0, 0, p.Sq, p.Sk),
-                                          kv_tiles_for<CAUSAL>(q0, 1, p.Sq, p.Sk));
+                    const Unit w = decode_unit<CAUSAL>(u, p);
+                    const int q0 = w.qp * ROWS_PER_CTA;
+                    const int bh = w.bh;
+                    const int n_max = max(w.n[0], w.n[1]);
+                    if (n_max == 0) continue;  // nothing to load (the MMA skips it too)
                     // Q_0, Q_1 are free once the previous unit's S MMAs completed
                     if (!(ok = wait_bounded(ctx, B_QE, (nu & 1) ^ 1))) break;
                     if (load_q) {
@@ -629,13 +679,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ptx::mbar_arrive_expect_tx(B_KF(s), L::TILE_BYTES);
                         for (int c = 0; c < L::NCH; ++c)
                             ptx::tma_load_3d(sK + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_k,
-                                             B_KF(s), c * CHUNK_ELEMS, j * BN, bh);
+                                             B_KF(s), c * CHUNK_ELEMS, (w.kv0 + j) * BN, bh);
                         last_k = pos;
                         if (!(ok = wait_bounded(ctx, B_VE(s), ph ^ 1))) break;
                         ptx::mbar_arrive_expect_tx(B_VF(s), L::TILE_BYTES);
                         for (int c = 0; c < L::NCH; ++c)
                             ptx::tma_load_3d(sV + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_v,
-                                             B_VF(s), c * CHUNK_ELEMS, j * BN, bh);
+                                             B_VF(s), c * CHUNK_ELEMS, (w.kv0 + j) * BN, bh);
                         last_v = pos;
                     }
                     kv += static_cast<uint32_t>(n_max);

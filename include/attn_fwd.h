@@ -32,6 +32,8 @@
 #ifndef ATTN_FWD_H
 #define ATTN_FWD_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -54,7 +56,8 @@ enum {
     ATTN_ERR_TIMEOUT = -8,   /* (status word) a pipeline wait ran out of time       */
     ATTN_ERR_SCALE = -9,     /* scale is NaN or infinite                            */
     ATTN_ERR_ALIAS = -10,    /* o or lse overlaps q, k or v                         */
-    ATTN_ERR_DEVICE = -11    /* no CUDA device, or the current one is not sm_100    */
+    ATTN_ERR_DEVICE = -11,   /* no CUDA device, or the current one is not sm_100    */
+    ATTN_ERR_WORKSPACE = -12 /* split pass: workspace smaller than required         */
 };
 
 /*
@@ -87,6 +90,36 @@ int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                   void *q_dev, void *k_dev, void *v_dev, void *o_dev, float *lse_dev,
                   int B, int H, int Sq, int Sk, int D, int causal, float scale,
                   int dtype, attn_stream_t stream);
+
+/*
+ * attn_fwd_splitkv -- the same pass computed as n_splits independent KV ranges per
+ * (256-row query block, head), for shapes with few query rows and long key sequences
+ * (decoding): each range writes its own normalised partial O and log-sum-exp into
+ * `workspace` (fp32), and a second kernel merges them,
+ *     LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s,
+ * which is the whole-range softmax attention exactly (each range's weight is its share
+ * of the full normaliser; a range no key of which a row sees has LSE_s = -inf).  The
+ * pages describe the online-softmax rescaling this relies on; the split itself is this
+ * library's (no counterpart on the pages).
+ *   n_splits   1 .. 1024 ranges of ceil(ceil(Sk/128) / n_splits) 128-key tiles each
+ *              (trailing ranges may be empty); attn_fwd_splitkv_default_splits gives
+ *              about two units of work per SM
+ *   workspace  device, 256-byte aligned, at least attn_fwd_splitkv_workspace_bytes(B,
+ *              H, Sq, D, n_splits) bytes, caller-owned, not overlapping any argument;
+ *              its contents are scratch (overwritten each call)
+ * Other arguments, layouts and errors as attn_fwd; ATTN_ERR_WORKSPACE when the
+ * workspace is too small.  Two kernels are queued on `stream`.
+ */
+int attn_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                     int B, int H, int Sq, int Sk, int D, int causal, float scale,
+                     int dtype, int n_splits, void *workspace, size_t workspace_bytes,
+                     attn_stream_t stream);
+
+/* Bytes of workspace attn_fwd_splitkv needs (0 for invalid arguments). */
+size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_splits);
+
+/* A split count giving about two units of work per SM of the current device. */
+int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk);
 
 /*
  * attn_fwd_status -- synchronise `stream`, copy the current device's status word

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_strerror():
     assert af.abi_version() == 1
-    for code in range(0, -12, -1):
+    for code in range(0, -13, -1):
         msg = af.strerror(code)
         assert msg and msg != "unknown error code", code
     assert af.strerror(12345) == "unknown error code"
@@ -98,3 +98,50 @@ def test_binding_rejects_bad_tensors():
         af.attention(q, q, q)
     with pytest.raises(ValueError):
         af.attention(q[0], q[0], q[0])
+
+
+W = 0x60000000  # fake 256-byte aligned workspace address
+
+
+def split_call(n_splits=4, ws=W, ws_bytes=None, **kw):
+    args = dict(q=Q, k=K, v=V, o=O, lse=L, B=1, H=2, Sq=64, Sk=4096, D=128, causal=0,
+                scale=0.1, dtype=af.ATTN_BF16)
+    args.update(kw)
+    if ws_bytes is None:
+        ws_bytes = af.splitkv_workspace_bytes(args["B"], args["H"], args["Sq"], args["D"],
+                                              max(n_splits, 1))
+    return af.attn_fwd_splitkv(args["q"], args["k"], args["v"], args["o"], args["lse"],
+                               args["B"], args["H"], args["Sq"], args["Sk"], args["D"],
+                               args["causal"], args["scale"], args["dtype"], n_splits, ws,
+                               ws_bytes, None)
+
+
+def test_splitkv_workspace_size_formula():
+    # partial O (fp32, rounded up to 256 bytes) then partial LSE (fp32)
+    B, H, Sq, D, S = 2, 3, 17, 64, 5
+    o_part = -(-(S * B * H * Sq * D * 4) // 256) * 256
+    assert af.splitkv_workspace_bytes(B, H, Sq, D, S) == o_part + S * B * H * Sq * 4
+    assert af.splitkv_workspace_bytes(B, H, Sq, 96, S) == 0
+    assert af.splitkv_workspace_bytes(B, H, Sq, D, 0) == 0
+    assert af.splitkv_workspace_bytes(B, H, Sq, D, 1025) == 0
+
+
+def test_splitkv_default_splits_in_range():
+    s = af.splitkv_default_splits(1, 8, 16, 32768)
+    assert 1 <= s <= 256
+    assert af.splitkv_default_splits(1, 1, 1, 100) == 1      # a single KV tile
+    assert af.splitkv_default_splits(0, 1, 1, 100) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_splits=0), af.ATTN_ERR_SHAPE),
+    (dict(n_splits=1025), af.ATTN_ERR_SHAPE),
+    (dict(ws=None), af.ATTN_ERR_NULLPTR),
+    (dict(ws=W + 128), af.ATTN_ERR_ALIGN),
+    (dict(ws_bytes=1024), af.ATTN_ERR_WORKSPACE),
+    (dict(ws=Q + 4096), af.ATTN_ERR_ALIAS),
+    (dict(ws=O - 256), af.ATTN_ERR_ALIAS),
+    (dict(D=80), af.ATTN_ERR_HEADDIM),
+])
+def test_splitkv_argument_errors(kw, code):
+    assert split_call(**kw) == code
