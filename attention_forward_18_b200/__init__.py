@@ -60,7 +60,7 @@ _lib.attn_fwd_splitkv.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _i, _i, _vp, ctypes
 _lib.attn_fwd_splitkv.restype = _i
 _lib.attn_fwd_splitkv_workspace_bytes.argtypes = [_i] * 5
 _lib.attn_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
-_lib.attn_fwd_splitkv_default_splits.argtypes = [_i] * 4
+_lib.attn_fwd_splitkv_default_splits.argtypes = [_i] * 5
 _lib.attn_fwd_splitkv_default_splits.restype = _i
 _lib.attn_fwd_status.argtypes = [_vp, ctypes.POINTER(_i)]
 _lib.attn_fwd_status.restype = _i
@@ -120,8 +120,8 @@ def splitkv_workspace_bytes(B, H, Sq, D, n_splits):
     return _lib.attn_fwd_splitkv_workspace_bytes(B, H, Sq, D, n_splits)
 
 
-def splitkv_default_splits(B, H, Sq, Sk):
-    return _lib.attn_fwd_splitkv_default_splits(B, H, Sq, Sk)
+def splitkv_default_splits(B, H, Sq, Sk, causal=False):
+    return _lib.attn_fwd_splitkv_default_splits(B, H, Sq, Sk, int(bool(causal)))
 
 
 def attn_fwd_status(stream=None):
@@ -199,7 +199,7 @@ def attention_splitkv(q, k, v, causal=False, scale=None, n_splits=None, out=None
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if n_splits is None:
-        n_splits = splitkv_default_splits(B, H, Sq, Sk)
+        n_splits = splitkv_default_splits(B, H, Sq, Sk, causal)
     nbytes = splitkv_workspace_bytes(B, H, Sq, D, n_splits)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)

@@ -316,18 +316,32 @@ size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_split
     return ws_bytes(B, H, Sq, D, n_splits);
 }
 
-int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk) {
+int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal) {
     if (B < 1 || H < 1 || Sq < 1 || Sk < 1) return 0;
     int num_sms = 0;
     if (check_device(&num_sms) != ATTN_OK) num_sms = 148;
     const int64_t units = static_cast<int64_t>((Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA) *
                           B * H;
-    const int n_kv = (Sk + attn::BN - 1) / attn::BN;
-    // about two units per SM, at least one KV tile per range
-    int64_t s = (2 * static_cast<int64_t>(num_sms) + units - 1) / units;
-    if (s > n_kv) s = n_kv;
-    if (s > kMaxSplits) s = kMaxSplits;
-    return s < 1 ? 1 : static_cast<int>(s);
+    // with the top-left causal mask no row sees a key past min(Sq, Sk)
+    const int keys = causal ? (Sq < Sk ? Sq : Sk) : Sk;
+    const int n_kv = (keys + attn::BN - 1) / attn::BN;
+    // Persistent CTAs take units round-robin, so the pass lasts about
+    //   ceil(units * n / SMs) rounds x (tiles per range + a fill of ~2 tiles);
+    // take the n with the least of that (the fewest splits among equals: less to merge).
+    int best = 1;
+    int64_t best_cost = INT64_MAX;
+    const int n_hi = n_kv < kMaxSplits ? n_kv : kMaxSplits;
+    for (int n = 1; n <= n_hi; ++n) {
+        const int chunk = (n_kv + n - 1) / n;
+        if ((n_kv + chunk - 1) / chunk != n) continue;  // some range would be empty
+        const int64_t rounds = (units * n + num_sms - 1) / num_sms;
+        const int64_t cost = rounds * (chunk + 2);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = n;
+        }
+    }
+    return best;
 }
 
 int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,

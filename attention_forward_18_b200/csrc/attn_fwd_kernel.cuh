@@ -167,11 +167,11 @@ struct Unit {
     int n[2];
 };
 
-template <bool CAUSAL>
+template <bool CAUSAL, bool SPLIT>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     Unit w;
-    w.split = u % p.n_splits;
-    const int rest = u / p.n_splits;
+    w.split = SPLIT ? u % p.n_splits : 0;
+    const int rest = SPLIT ? u / p.n_splits : u;
     if constexpr (CAUSAL) {
         w.qp = p.n_qp - 1 - rest / p.BH;
         w.bh = rest % p.BH;
@@ -180,8 +180,8 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
         w.bh = rest / p.n_qp;
     }
     const int n_all = (p.Sk + BN - 1) / BN;
-    w.kv0 = w.split * p.chunk_tiles;
-    const int kv_end = min(n_all, w.kv0 + p.chunk_tiles);
+    w.kv0 = SPLIT ? w.split * p.chunk_tiles : 0;
+    const int kv_end = SPLIT ? min(n_all, w.kv0 + p.chunk_tiles) : n_all;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int first = w.qp * ROWS_PER_CTA + BM * t;
@@ -265,9 +265,7 @@ __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, 
         alpha = ptx::ex2(m_used - m_tile);
         m_used = m_tile;
     }
-    // a row with no visible key so far (possible in a KV range of a split pass) keeps
-    // m = -inf; its p are 0 and nothing may compute -inf - (-inf)
-    const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+    const float neg_m = -m_used;
 
     // p = 2^(s * c - m): scale and shift in one packed fma per column pair; the row
     // sum accumulates in a packed pair too
@@ -409,7 +407,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int u = unit_of(r, n_units);
             if (u < 0) break;
-            const Unit w = decode_unit<CAUSAL>(u, p);
+            const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
             const int q0t = w.qp * ROWS_PER_CTA + BM * t;
             const int qrow = q0t + row;
             const int n_t = w.n[t];
@@ -459,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int u = unit_of(r, n_units);
             if (u < 0) break;
-            const Unit w = decode_unit<CAUSAL>(u, p);
+            const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
             const int64_t head_row = static_cast<int64_t>(w.split) * p.BH + w.bh;
             for (int t = 0; ok && t < 2; ++t) {
                 const int qrow = w.qp * ROWS_PER_CTA + BM * t + row;
@@ -595,7 +593,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
-                    const Unit w = decode_unit<CAUSAL>(u, p);
+                    const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
                     const int n_t[2] = {w.n[0], w.n[1]};
                     const int n_max = max(n_t[0], n_t[1]);
                     if (n_max == 0) continue;  // a split range no query row of the unit sees
@@ -655,7 +653,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
-                    const Unit w = decode_unit<CAUSAL>(u, p);
+                    const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
                     const int q0 = w.qp * ROWS_PER_CTA;
                     const int bh = w.bh;
                     const int n_max = max(w.n[0], w.n[1]);

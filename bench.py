@@ -20,8 +20,8 @@ Also reported: `e2e` (the same steps through attn_fwd_host from pinned host buff
 copies included), `roofline` (the dominant kernel's achieved TFLOP/s against the
 measured dense bf16 peak), `cpu_baseline` (the fp64 CPU oracle on a bounded sample
 of the workload, rank 0 at N=1), `clocks` (NVML samples taken during the timed
-region) and `extra` (the other large workloads, timed the same way, outside the
-timed region).
+region) and `extra` (the other large workloads, and the split-KV pass on
+decode-shaped workloads, timed the same way, outside the timed region).
 """
 import argparse
 import json
@@ -376,6 +376,57 @@ def extra_workloads(af_names, world):
     return res
 
 
+def decode_workloads(names):
+    """The split-KV pass on decode-shaped workloads (HBM-bound: K and V are read once,
+    the score work is small), timed like the rest with a cold L2; the whole pass on the
+    same tensors beside it."""
+    import attention_forward_18_b200 as af
+    from workloads import DECODE_WORKLOADS
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    res = {}
+    for name in names:
+        w = DECODE_WORKLOADS[name]
+        q, k, v = (t.to(dev) for t in make_inputs(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+        dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
+        n = af.splitkv_default_splits(w.B, w.H, w.Sq, w.Sk, False)
+        nbytes = af.splitkv_workspace_bytes(w.B, w.H, w.Sq, w.D, n)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                w.B, w.H, w.Sq, w.Sk, w.D, 0, w.scale, dcode)
+
+        def split():
+            rc = af.attn_fwd_splitkv(*args, n, ws.data_ptr(), nbytes, stream.cuda_stream)
+            if rc != 0:
+                raise af.AttnError(rc, "attn_fwd_splitkv")
+
+        def whole():
+            rc = af.attn_fwd(*args, stream.cuda_stream)
+            if rc != 0:
+                raise af.AttnError(rc, "attn_fwd")
+        ms = statistics.median(x[0] for x in time_steps([split], 20, 5, flush, stream))
+        ms_whole = statistics.median(x[0] for x in time_steps([whole], 10, 3, flush, stream))
+        gbs = w.io_bytes() / (ms * 1e-3) / 1e9
+        res[name] = {
+            "shape": f"B={w.B} H={w.H} Sq={w.Sq} Sk={w.Sk} D={w.D} {w.dtype}",
+            "n_splits": n, "ms": round(ms, 4), "GB/s": round(gbs, 1),
+            "frac_of_hbm": round(gbs / hbm, 4),
+            "TFLOP/s": round(w.flops(False) / (ms * 1e-3) / 1e12, 1),
+            "whole_pass_GB/s": round(w.io_bytes() / (ms_whole * 1e-3) / 1e9, 1)}
+        status = af.attn_fwd_status(stream)
+        if status != 0:
+            raise af.AttnError(status, f"device status after {name}")
+        del q, k, v, o, lse, ws
+        torch.cuda.empty_cache()
+    res["peak_GB/s"] = f"{hbm} ({peak_kind} HBM copy)"
+    return res
+
+
 # ---------------------------------------------------------------- oracle (CPU) arm
 def oracle_sample(w, seconds, max_heads=None):
     """Time the fp64 CPU oracle as it stands on whole heads of the workload (every
@@ -472,6 +523,7 @@ def main():
         line = cuda_arm(args, world, rank, local)
         if rank == 0 and not args.no_extra:
             line["extra"] = extra_workloads(["C3", "C4", "C5"], world)
+            line["extra"]["decode_splitkv"] = decode_workloads(["DEC1", "DEC2", "DEC3", "DEC4"])
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             w = WORKLOADS[args.workload]
             tf, cores, desc = oracle_sample(w, args.cpu_seconds)

@@ -102,8 +102,8 @@ int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
  * pages describe the online-softmax rescaling this relies on; the split itself is this
  * library's (no counterpart on the pages).
  *   n_splits   1 .. 1024 ranges of ceil(ceil(Sk/128) / n_splits) 128-key tiles each
- *              (trailing ranges may be empty); attn_fwd_splitkv_default_splits gives
- *              about two units of work per SM
+ *              (trailing ranges may be empty); attn_fwd_splitkv_default_splits picks
+ *              one for the device
  *   workspace  device, 256-byte aligned, at least attn_fwd_splitkv_workspace_bytes(B,
  *              H, Sq, D, n_splits) bytes, caller-owned, not overlapping any argument;
  *              its contents are scratch (overwritten each call)
@@ -118,8 +118,9 @@ int attn_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float
 /* Bytes of workspace attn_fwd_splitkv needs (0 for invalid arguments). */
 size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_splits);
 
-/* A split count giving about two units of work per SM of the current device. */
-int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk);
+/* A split count for these sizes on the current device: the one that balances
+ * (query block, head, range) units over the SMs best (1 .. 1024; 0 for invalid sizes). */
+int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal);
 
 /*
  * attn_fwd_status -- synchronise `stream`, copy the current device's status word

@@ -127,10 +127,17 @@ def test_splitkv_workspace_size_formula():
 
 
 def test_splitkv_default_splits_in_range():
+    # no device here: the library assumes 148 SMs
     s = af.splitkv_default_splits(1, 8, 16, 32768)
     assert 1 <= s <= 256
     assert af.splitkv_default_splits(1, 1, 1, 100) == 1      # a single KV tile
     assert af.splitkv_default_splits(0, 1, 1, 100) == 0
+    # 16 heads x 1024 tiles: one round of 144 units of 114 tiles beats two rounds
+    assert af.splitkv_default_splits(2, 8, 1, 131072) == 9
+    # top-left causal with one query row: only key 0 is visible, nothing to split
+    assert af.splitkv_default_splits(1, 8, 1, 131072, causal=True) == 1
+    # many units already fill the SMs
+    assert af.splitkv_default_splits(64, 32, 256, 256) == 1
 
 
 @pytest.mark.parametrize("kw,code", [

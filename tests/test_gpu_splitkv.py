@@ -115,3 +115,23 @@ def test_workspace_too_small_is_rejected_on_device():
                              1, 2, 8, 3000, 128, 0, 0.1, af.ATTN_BF16, 4, ws.data_ptr(),
                              need - 1, None)
     assert rc == af.ATTN_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("name", ["DEC1", "DEC2", "DEC3", "DEC4"])
+def test_decode_workloads_in_bench_configuration(name):
+    """The benchmark's decode workloads with the split count the benchmark uses: every
+    row against the oracle (sampled rows for DEC3's 2048 rows x 64K keys)."""
+    from workloads import DECODE_WORKLOADS, make_inputs, sample_rows
+    w = DECODE_WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    n = af.splitkv_default_splits(w.B, w.H, w.Sq, w.Sk, False)
+    o, lse = run_split(q, k, v, False, w.scale, n)
+    qd, kd, vd = q.double().numpy(), k.double().numpy(), v.double().numpy()
+    if w.Sq <= 8:
+        o_ref, lse_ref = oracle.attn_ref(qd, kd, vd, False, w.scale)
+        compare(o, lse, o_ref, lse_ref, name)
+    else:
+        rows = sample_rows(w.B, w.H, w.Sq, 64, seed=w.seed)
+        ro, rl = oracle.attn_ref_rows(qd, kd, vd, rows, False, w.scale)
+        idx = tuple(np.array(rows).T)
+        compare(o[idx], lse[idx], ro, rl, name)

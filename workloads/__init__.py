@@ -63,6 +63,19 @@ WORKLOADS = {
                    note="long-context causal"),
 }
 
+# Decode-shaped workloads of the split-KV pass: few query rows per head against a long
+# key sequence (the regime the pages' decode kernel serves), same input recipe.
+DECODE_WORKLOADS = {
+    "DEC1": Workload("DEC1", 1, 32, 1, 32768, 128, "bf16", (False,), 5,
+                     note="one sequence, one query row per head, 32K keys"),
+    "DEC2": Workload("DEC2", 8, 32, 1, 8192, 128, "bf16", (False,), 6,
+                     note="batch of 8 sequences, one query row per head, 8K keys"),
+    "DEC3": Workload("DEC3", 2, 16, 64, 65536, 128, "bf16", (False,), 7,
+                     note="64 query rows per head (a block of drafted tokens), 64K keys"),
+    "DEC4": Workload("DEC4", 16, 32, 1, 4096, 64, "f16", (False,), 8,
+                     note="batch of 16, D=64, 4K keys"),
+}
+
 
 def flops(B, H, Sq, Sk, D, causal):
     """Counted FLOPs of one pass: 4*B*H*Sq*Sk*D (two GEMMs of 2 flops per
