@@ -10,8 +10,13 @@ softmax-attention definition that the TileLang tutorial's FlashAttention section
 validates against (pro.edgex.exchange summary, FlashAttention paragraph; datastack.it,
 "Cosa copre il tutorial": causal and non-causal):
 
-    O = softmax(scale * Q K^T  [+ top-left causal mask]) V
+    O = softmax(scale * Q K^T  [+ causal mask]) V
     LSE_i = ln sum_j exp(scale * q_i . k_j)     (over the unmasked j)
+
+The causal mask is top-left aligned (key j visible to query i iff j <= i) unless
+``mask=CAUSAL_BOTTOM_RIGHT`` (j <= i + Sk - Sq; a row that sees no key gets O = 0,
+LSE = -inf).  K and V may have fewer heads than Q (``Hkv`` divides ``H``; query head
+h reads K/V head h // (H // Hkv)).  Both are the library's options beyond the pages.
 
 Pins (see tests/test_oracle_pins.py): closed forms (Sk = 1, Q = 0, constant V,
 causal row 0, one-hot attention), invariants (row sums, permutation and shift
@@ -23,6 +28,10 @@ import os
 import numpy as np
 
 from . import build as _build
+
+NO_MASK = 0
+CAUSAL_TOP_LEFT = 1
+CAUSAL_BOTTOM_RIGHT = 2
 
 ORACLE_OK = 0
 ORACLE_ERR_ARGS = 1
@@ -43,6 +52,13 @@ def _bind(path):
                                       dp, dp, lp, lp, lp, lp, lp, ctypes.c_int,
                                       ctypes.c_double]
     lib.attn_ref_rows_f64.restype = ctypes.c_int
+    lib.attn_ref_ex_f64.argtypes = [dp, dp, dp, dp, dp, dp, lp, lp, lp, lp, lp, lp,
+                                    ctypes.c_int, ctypes.c_double]
+    lib.attn_ref_ex_f64.restype = ctypes.c_int
+    lib.attn_ref_rows_ex_f64.argtypes = [dp, dp, dp, ctypes.POINTER(ctypes.c_int64), lp,
+                                         dp, dp, lp, lp, lp, lp, lp, lp, ctypes.c_int,
+                                         ctypes.c_double]
+    lib.attn_ref_rows_ex_f64.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -112,4 +128,53 @@ def attn_ref_rows(q, k, v, rows, causal, scale, lib=None):
     return o, lse
 
 
-__all__ = ["attn_ref", "attn_ref_rows", "load", "num_threads"]
+def _mask_code(causal, mask):
+    if mask is not None:
+        if mask not in (NO_MASK, CAUSAL_TOP_LEFT, CAUSAL_BOTTOM_RIGHT):
+            raise ValueError(f"unknown mask {mask}")
+        return int(mask)
+    return CAUSAL_TOP_LEFT if causal else NO_MASK
+
+
+def attn_ref_ex(q, k, v, mask=None, scale=1.0, causal=False, return_probs=False, lib=None):
+    """Whole problem with the extended options: k, v [B,Hkv,Sk,D] with Hkv dividing
+    q's H; `mask` one of NO_MASK, CAUSAL_TOP_LEFT, CAUSAL_BOTTOM_RIGHT (or None: taken
+    from `causal`).  Returns (O, LSE[, P]) in fp64 like attn_ref."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, Sk, D) or v.shape != (B, Hkv, Sk, D):
+        raise ValueError("k and v must be [B,Hkv,Sk,D] with q's B and D")
+    o = np.empty((B, H, Sq, D), dtype=np.float64)
+    lse = np.empty((B, H, Sq), dtype=np.float64)
+    p = np.empty((B, H, Sq, Sk), dtype=np.float64) if return_probs else None
+    rc = lib.attn_ref_ex_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                             _ptr(p) if p is not None else None,
+                             B, H, Hkv, Sq, Sk, D, _mask_code(causal, mask), float(scale))
+    if rc != ORACLE_OK:
+        raise RuntimeError(f"oracle attn_ref_ex_f64 failed with code {rc}")
+    return (o, lse, p) if return_probs else (o, lse)
+
+
+def attn_ref_rows_ex(q, k, v, rows, mask=None, scale=1.0, causal=False, lib=None):
+    """Selected rows with the extended options (see attn_ref_ex)."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Sq, D = q.shape
+    Hkv, Sk = k.shape[1], k.shape[2]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = lib.attn_ref_rows_ex_f64(_ptr(q), _ptr(k), _ptr(v),
+                                  rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n,
+                                  _ptr(o), _ptr(lse), B, H, Hkv, Sq, Sk, D,
+                                  _mask_code(causal, mask), float(scale))
+    if rc != ORACLE_OK:
+        raise RuntimeError(f"oracle attn_ref_rows_ex_f64 failed with code {rc}")
+    return o, lse
+
+
+__all__ = ["attn_ref", "attn_ref_rows", "attn_ref_ex", "attn_ref_rows_ex", "load",
+           "num_threads", "NO_MASK", "CAUSAL_TOP_LEFT", "CAUSAL_BOTTOM_RIGHT"]

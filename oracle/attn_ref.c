@@ -11,7 +11,9 @@
  * fusion:
  *
  *   s_ij   = scale * sum_d Q[i,d] K[j,d]                  scaled scores
- *   s_ij   = -inf         if causal and j > i             top-left causal mask
+ *   s_ij   = -inf         if causal and j > i + off       causal mask: off = 0 aligns
+ *                                                         it top-left, off = Sk - Sq
+ *                                                         bottom-right
  *   m_i    = max_j s_ij
  *   p_ij   = exp(s_ij - m_i) / sum_j exp(s_ij - m_i)      row softmax
  *   O[i,:] = sum_j p_ij V[j,:]
@@ -35,7 +37,14 @@
  * Each call checks, for every output row, that the softmax row sums to one within
  * 1e-12; a failed check returns ORACLE_ERR_ROWSUM.
  *
- * Layouts: Q [B,H,Sq,D], K and V [B,H,Sk,D], O [B,H,Sq,D], LSE [B,H,Sq], all
+ * Extensions of the same definition (the pages name only causal and non-causal; these
+ * are this library's options, written out the same plain way):
+ *   - bottom-right causal alignment (off = Sk - Sq: the last query row sees every
+ *     key); with Sq > Sk the first Sq - Sk rows then see no key at all, and such a
+ *     row is defined as O = 0, LSE = -inf (the empty sum);
+ *   - grouped K/V heads: Hkv divides H, query head h reads K/V head h / (H / Hkv).
+ *
+ * Layouts: Q [B,H,Sq,D], K and V [B,Hkv,Sk,D], O [B,H,Sq,D], LSE [B,H,Sq], all
  * contiguous row-major fp64.  Threads: OpenMP over heads (full entry point) or over
  * rows (row entry point).
  */
@@ -47,6 +56,9 @@
 #ifdef _OPENMP
 #include <omp.h>
 #endif
+
+/* mask argument */
+enum { ORACLE_NO_MASK = 0, ORACLE_CAUSAL_TOP_LEFT = 1, ORACLE_CAUSAL_BOTTOM_RIGHT = 2 };
 
 enum {
     ORACLE_OK = 0,
@@ -72,7 +84,7 @@ int oracle_num_threads(void)
  * Returns ORACLE_OK or ORACLE_ERR_ROWSUM.
  */
 static int attend_one_row(const double *q_i, const double *kh, const double *vh,
-                          long i, long Sk, long D, int causal, double scale,
+                          long i, long Sq, long Sk, long D, int mask, double scale,
                           double *srow, double *o_i, double *lse_i)
 {
     /* scores, then the causal mask */
@@ -82,8 +94,9 @@ static int attend_one_row(const double *q_i, const double *kh, const double *vh,
             dot += q_i[d] * kh[j * D + d];
         srow[j] = scale * dot;
     }
-    if (causal) {
-        for (long j = i + 1; j < Sk; ++j)
+    if (mask != ORACLE_NO_MASK) {
+        const long off = (mask == ORACLE_CAUSAL_BOTTOM_RIGHT) ? Sk - Sq : 0;
+        for (long j = (i + 1 + off > 0 ? i + 1 + off : 0); j < Sk; ++j)
             srow[j] = -INFINITY;
     }
 
@@ -92,6 +105,15 @@ static int attend_one_row(const double *q_i, const double *kh, const double *vh,
     for (long j = 0; j < Sk; ++j)
         if (srow[j] > m)
             m = srow[j];
+    if (m == -INFINITY) {
+        /* no visible key: the empty sum (no weights, O = 0, LSE = ln 0) */
+        for (long j = 0; j < Sk; ++j)
+            srow[j] = 0.0;
+        for (long d = 0; d < D; ++d)
+            o_i[d] = 0.0;
+        *lse_i = -INFINITY;
+        return ORACLE_OK;
+    }
     double l = 0.0;
     for (long j = 0; j < Sk; ++j) {
         srow[j] = exp(srow[j] - m);
@@ -118,9 +140,16 @@ static int attend_one_row(const double *q_i, const double *kh, const double *vh,
     return ORACLE_OK;
 }
 
-static int shape_ok(long B, long H, long Sq, long Sk, long D)
+static int shape_ok(long B, long H, long Hkv, long Sq, long Sk, long D, int mask)
 {
-    return B >= 1 && H >= 1 && Sq >= 1 && Sk >= 1 && D >= 1;
+    return B >= 1 && H >= 1 && Hkv >= 1 && H % Hkv == 0 && Sq >= 1 && Sk >= 1 && D >= 1 &&
+           mask >= ORACLE_NO_MASK && mask <= ORACLE_CAUSAL_BOTTOM_RIGHT;
+}
+
+/* Index of the K/V head that query head h of batch b reads. */
+static long kv_head(long b, long h, long H, long Hkv)
+{
+    return b * Hkv + h / (H / Hkv);
 }
 
 /*
@@ -128,12 +157,12 @@ static int shape_ok(long B, long H, long Sq, long Sk, long D)
  * masked, softmaxed row by row, and multiplied by V.
  * p_out (nullable) receives the probability matrices, [B,H,Sq,Sk].
  */
-int attn_ref_f64(const double *q, const double *k, const double *v,
-                 double *o, double *lse, double *p_out,
-                 long B, long H, long Sq, long Sk, long D,
-                 int causal, double scale)
+int attn_ref_ex_f64(const double *q, const double *k, const double *v,
+                    double *o, double *lse, double *p_out,
+                    long B, long H, long Hkv, long Sq, long Sk, long D,
+                    int mask, double scale)
 {
-    if (!q || !k || !v || !o || !lse || !shape_ok(B, H, Sq, Sk, D))
+    if (!q || !k || !v || !o || !lse || !shape_ok(B, H, Hkv, Sq, Sk, D, mask))
         return ORACLE_ERR_ARGS;
 
     const long heads = B * H;
@@ -151,10 +180,11 @@ int attn_ref_f64(const double *q, const double *k, const double *v,
             if (!smat)
                 continue;
             const double *qh = q + bh * Sq * D;
-            const double *kh = k + bh * Sk * D;
-            const double *vh = v + bh * Sk * D;
+            const long kvh = kv_head(bh / H, bh % H, H, Hkv);
+            const double *kh = k + kvh * Sk * D;
+            const double *vh = v + kvh * Sk * D;
             for (long i = 0; i < Sq; ++i) {
-                int rc = attend_one_row(qh + i * D, kh, vh, i, Sk, D, causal, scale,
+                int rc = attend_one_row(qh + i * D, kh, vh, i, Sq, Sk, D, mask, scale,
                                         smat + i * Sk, o + (bh * Sq + i) * D,
                                         lse + bh * Sq + i);
                 if (rc != ORACLE_OK) {
@@ -170,17 +200,28 @@ int attn_ref_f64(const double *q, const double *k, const double *v,
     return status;
 }
 
+/* The original entry point: K/V heads = query heads, causal = top-left. */
+int attn_ref_f64(const double *q, const double *k, const double *v,
+                 double *o, double *lse, double *p_out,
+                 long B, long H, long Sq, long Sk, long D,
+                 int causal, double scale)
+{
+    return attn_ref_ex_f64(q, k, v, o, lse, p_out, B, H, H, Sq, Sk, D,
+                           causal ? ORACLE_CAUSAL_TOP_LEFT : ORACLE_NO_MASK, scale);
+}
+
 /*
  * Selected rows only (the same definition restricted to the requested query rows,
  * for spot checks of problems too large to run whole).
  * rows: n triples (b, h, i).  o: n x D, lse: n.
  */
-int attn_ref_rows_f64(const double *q, const double *k, const double *v,
-                      const int64_t *rows, long n, double *o, double *lse,
-                      long B, long H, long Sq, long Sk, long D,
-                      int causal, double scale)
+int attn_ref_rows_ex_f64(const double *q, const double *k, const double *v,
+                         const int64_t *rows, long n, double *o, double *lse,
+                         long B, long H, long Hkv, long Sq, long Sk, long D,
+                         int mask, double scale)
 {
-    if (!q || !k || !v || !rows || !o || !lse || n < 0 || !shape_ok(B, H, Sq, Sk, D))
+    if (!q || !k || !v || !rows || !o || !lse || n < 0 ||
+        !shape_ok(B, H, Hkv, Sq, Sk, D, mask))
         return ORACLE_ERR_ARGS;
     for (long r = 0; r < n; ++r) {
         if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 ||
@@ -201,9 +242,10 @@ int attn_ref_rows_f64(const double *q, const double *k, const double *v,
             if (!srow)
                 continue;
             const long bh = rows[3 * r] * H + rows[3 * r + 1];
+            const long kvh = kv_head(rows[3 * r], rows[3 * r + 1], H, Hkv);
             const long i = rows[3 * r + 2];
-            int rc = attend_one_row(q + (bh * Sq + i) * D, k + bh * Sk * D, v + bh * Sk * D,
-                                    i, Sk, D, causal, scale, srow, o + r * D, lse + r);
+            int rc = attend_one_row(q + (bh * Sq + i) * D, k + kvh * Sk * D, v + kvh * Sk * D,
+                                    i, Sq, Sk, D, mask, scale, srow, o + r * D, lse + r);
             if (rc != ORACLE_OK) {
 #pragma omp atomic write
                 status = rc;
@@ -212,4 +254,13 @@ int attn_ref_rows_f64(const double *q, const double *k, const double *v,
         free(srow);
     }
     return status;
+}
+
+int attn_ref_rows_f64(const double *q, const double *k, const double *v,
+                      const int64_t *rows, long n, double *o, double *lse,
+                      long B, long H, long Sq, long Sk, long D,
+                      int causal, double scale)
+{
+    return attn_ref_rows_ex_f64(q, k, v, rows, n, o, lse, B, H, H, Sq, Sk, D,
+                                causal ? ORACLE_CAUSAL_TOP_LEFT : ORACLE_NO_MASK, scale);
 }

@@ -224,7 +224,75 @@ def pin_rows_match_whole(lib):
             assert rl[n] == lse[b, h, i]
 
 
+def pin_bottom_right_closed_forms(lib):
+    """Bottom-right causal mask: query i sees keys 0 .. i + Sk - Sq.  With Q = 0 the
+    visible weights are uniform, so O is the mean of those V rows and LSE = ln(count);
+    with Sq > Sk the first Sq - Sk rows see nothing: O = 0, LSE = -inf (empty sum);
+    with Sq = Sk it is the top-left mask (row i sees 0..i)."""
+    for (Sq, Sk) in ((5, 9), (7, 3), (6, 6)):
+        B, H, D = 1, 2, 4
+        q = np.zeros((B, H, Sq, D))
+        k, v = _rand((B, H, Sk, D), 40 + Sq), _rand((B, H, Sk, D), 50 + Sk)
+        o, lse = oracle.attn_ref_ex(q, k, v, oracle.CAUSAL_BOTTOM_RIGHT, 0.5, lib=lib)
+        for i in range(Sq):
+            last = i + Sk - Sq          # last visible key
+            if last < 0:
+                assert (o[:, :, i, :] == 0.0).all()
+                assert (lse[:, :, i] == -np.inf).all()
+            else:
+                np.testing.assert_allclose(o[:, :, i, :], v[:, :, : last + 1, :].mean(axis=2),
+                                           rtol=0, atol=1e-14)
+                np.testing.assert_allclose(lse[:, :, i], math.log(last + 1), rtol=0, atol=1e-14)
+
+
+def pin_bottom_right_torch(lib):
+    """PyTorch's float64 math SDPA with an explicit lower-right boolean mask
+    (torch.tril with diagonal Sk - Sq) and torch.logsumexp of the masked scores;
+    Sq <= Sk so no row is empty."""
+    for (Sq, Sk, seed) in ((3, 11, 60), (17, 40, 61), (9, 9, 62)):
+        B, H, D = 2, 3, 8
+        q, k, v = _rand((B, H, Sq, D), seed), _rand((B, H, Sk, D), seed + 1), _rand((B, H, Sk, D), seed + 2)
+        scale = 0.3
+        o, lse = oracle.attn_ref_ex(q, k, v, oracle.CAUSAL_BOTTOM_RIGHT, scale, lib=lib)
+        tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+        allowed = torch.tril(torch.ones(Sq, Sk, dtype=torch.bool), diagonal=Sk - Sq)
+        with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed,
+                                                                   scale=scale)
+        np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+        s = scale * torch.einsum("bhid,bhjd->bhij", tq, tk)
+        s = s.masked_fill(~allowed, float("-inf"))
+        np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def pin_grouped_heads_torch(lib):
+    """K/V with fewer heads than Q: PyTorch's SDPA with enable_gqa (query head h reads
+    K/V head h // (H // Hkv)), and the LSE of K expanded with repeat_interleave."""
+    B, H, Hkv, Sq, Sk, D = 2, 8, 2, 6, 13, 8
+    q, k, v = _rand((B, H, Sq, D), 70), _rand((B, Hkv, Sk, D), 71), _rand((B, Hkv, Sk, D), 72)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    for causal in (False, True):
+        o, lse = oracle.attn_ref_ex(q, k, v, None, 0.4, causal=causal, lib=lib)
+        with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                tq, tk, tv, is_causal=causal, scale=0.4, enable_gqa=True)
+        np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+        ke = tk.repeat_interleave(H // Hkv, dim=1)
+        s = 0.4 * torch.einsum("bhid,bhjd->bhij", tq, ke)
+        if causal:
+            s = s.masked_fill(~torch.tril(torch.ones(Sq, Sk, dtype=torch.bool)), float("-inf"))
+        np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-12)
+    # the row entry point follows the same head mapping and mask
+    rows = [(0, 7, 5), (1, 3, 0), (1, 4, 2)]
+    for mask in (oracle.NO_MASK, oracle.CAUSAL_TOP_LEFT, oracle.CAUSAL_BOTTOM_RIGHT):
+        o, lse = oracle.attn_ref_ex(q, k, v, mask, 0.4, lib=lib)
+        ro, rl = oracle.attn_ref_rows_ex(q, k, v, rows, mask, 0.4, lib=lib)
+        idx = tuple(np.array(rows).T)
+        assert np.array_equal(ro, o[idx]) and np.array_equal(rl, lse[idx])
+
+
 ALL_PINS = [pin_single_key, pin_zero_query, pin_constant_value, pin_causal_first_row,
             pin_hand_2x2, pin_hand_3x2_causal, pin_one_hot_huge_margin,
             pin_probability_rows, pin_permutation, pin_key_shift, pin_linear_in_value,
-            pin_torch_sdpa, pin_rows_match_whole]
+            pin_torch_sdpa, pin_rows_match_whole,
+            pin_bottom_right_closed_forms, pin_bottom_right_torch, pin_grouped_heads_torch]

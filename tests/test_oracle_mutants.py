@@ -12,16 +12,26 @@ from oracle import build as obuild
 from oracle_pins import ALL_PINS
 
 # (name, original text, replacement) -- each a mistake one could plausibly make.
+MASK_LOOP = "for (long j = (i + 1 + off > 0 ? i + 1 + off : 0); j < Sk; ++j)"
+OFFSET = "const long off = (mask == ORACLE_CAUSAL_BOTTOM_RIGHT) ? Sk - Sq : 0;"
+
+# (name, original text, replacement) -- each a mistake one could plausibly make.
 MUTANTS = [
     ("scale_dropped", "srow[j] = scale * dot;", "srow[j] = dot;"),
     ("score_sign", "srow[j] = scale * dot;", "srow[j] = -scale * dot;"),
-    ("mask_wrong_side", "for (long j = i + 1; j < Sk; ++j)",
-     "for (long j = 0; j < i && j < Sk; ++j)"),
-    ("mask_hides_diagonal", "for (long j = i + 1; j < Sk; ++j)", "for (long j = i; j < Sk; ++j)"),
-    ("mask_one_late", "for (long j = i + 1; j < Sk; ++j)", "for (long j = i + 2; j < Sk; ++j)"),
-    # bottom-right alignment (key j visible to query i when j <= i + Sk - Sq); the
-    # edit that threads Sq into the row routine is in _bottom_right_source
-    ("mask_bottom_right", "for (long j = i + 1; j < Sk; ++j)", None),
+    ("mask_wrong_side", MASK_LOOP, "for (long j = 0; j < i + off && j < Sk; ++j)"),
+    ("mask_hides_diagonal", MASK_LOOP,
+     "for (long j = (i + off > 0 ? i + off : 0); j < Sk; ++j)"),
+    ("mask_one_late", MASK_LOOP,
+     "for (long j = (i + 2 + off > 0 ? i + 2 + off : 0); j < Sk; ++j)"),
+    # bottom-right alignment applied to the top-left mode
+    ("mask_bottom_right", OFFSET, "const long off = Sk - Sq;"),
+    ("bottom_right_offset_sign", OFFSET,
+     "const long off = (mask == ORACLE_CAUSAL_BOTTOM_RIGHT) ? Sq - Sk : 0;"),
+    ("bottom_right_ignored", OFFSET, "const long off = 0;"),
+    ("empty_row_lse", "*lse_i = -INFINITY;\n        return ORACLE_OK;",
+     "*lse_i = 0.0;\n        return ORACLE_OK;"),
+    ("gqa_heads_modulo", "return b * Hkv + h / (H / Hkv);", "return b * Hkv + h % Hkv;"),
     ("no_max_subtraction", "srow[j] = exp(srow[j] - m);", "srow[j] = exp(srow[j]);"),
     ("lse_without_max", "*lse_i = m + log(l);", "*lse_i = log(l);"),
     ("lse_log2", "*lse_i = m + log(l);", "*lse_i = m + log2(l);"),
@@ -51,25 +61,10 @@ def _build_mutant(tmp_path, src, name):
     return oracle.load(str(out))
 
 
-def _bottom_right_source(src):
-    # the row routine does not see Sq: pass it through a file-scope variable
-    src = src.replace("static int attend_one_row(", "static long g_sq;\nstatic int attend_one_row(")
-    src = src.replace("if (causal) {\n        for (long j = i + 1; j < Sk; ++j)",
-                      "if (causal) {\n        long Sq = g_sq;\n        for (long j = (i + 1 + Sk - Sq > 0 ? i + 1 + Sk - Sq : 0); j < Sk; ++j)")
-    src = src.replace("const long heads = B * H;", "const long heads = B * H;\n    g_sq = Sq;")
-    src = src.replace("int status = ORACLE_OK;\n#pragma omp parallel\n    {\n        double *srow",
-                      "int status = ORACLE_OK;\n    g_sq = Sq;\n#pragma omp parallel\n    {\n        double *srow")
-    return src
-
-
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(tmp_path, original_source, name, old, new):
-    assert old in original_source, f"mutation anchor for {name} not found in the oracle"
-    if new is None:
-        src = _bottom_right_source(original_source)
-        assert src != original_source
-    else:
-        src = original_source.replace(old, new)
+    assert original_source.count(old) == 1, f"mutation anchor for {name} not found once"
+    src = original_source.replace(old, new)
     lib = _build_mutant(tmp_path, src, name)
     caught = []
     for pin in ALL_PINS:
