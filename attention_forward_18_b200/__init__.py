@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libattn_fwd.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m attention_forward_18_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python attention_forward_18_b200/build.py` "
         "(there is no non-CUDA implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)

@@ -1,6 +1,8 @@
 """Build the CUDA library libattn_fwd.so in-tree with nvcc for sm_100a.
 
-    python -m attention_forward_18_b200.build [--force] [--verbose-ptxas]
+    python attention_forward_18_b200/build.py [--force] [--verbose-ptxas]
+
+(run as a script: importing the package needs the library this builds)
 """
 import os
 import subprocess
