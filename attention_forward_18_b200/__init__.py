@@ -44,8 +44,11 @@ ATTN_ERR_WORKSPACE = -12
 
 # Every symbol include/attn_fwd.h declares.
 EXPORTS = ("attn_fwd", "attn_fwd_host", "attn_fwd_splitkv", "attn_fwd_splitkv_workspace_bytes",
-           "attn_fwd_splitkv_default_splits", "attn_fwd_status", "attn_fwd_strerror",
-           "attn_fwd_abi_version", "attn_fwd_debug")
+           "attn_fwd_splitkv_default_splits", "attn_fwd_splitkv_noalloc", "attn_fwd_status",
+           "attn_fwd_strerror", "attn_fwd_abi_version", "attn_fwd_debug")
+
+# Bytes of the library's own scratch behind attn_fwd_splitkv_noalloc.
+SPLITKV_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _SIZES = [_i] * 6 + [_f, _i, _vp]   # B, H, Sq, Sk, D, causal, scale, dtype, stream
@@ -62,6 +65,8 @@ _lib.attn_fwd_splitkv_workspace_bytes.argtypes = [_i] * 5
 _lib.attn_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
 _lib.attn_fwd_splitkv_default_splits.argtypes = [_i] * 5
 _lib.attn_fwd_splitkv_default_splits.restype = _i
+_lib.attn_fwd_splitkv_noalloc.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _i, _i, _vp]
+_lib.attn_fwd_splitkv_noalloc.restype = _i
 _lib.attn_fwd_status.argtypes = [_vp, ctypes.POINTER(_i)]
 _lib.attn_fwd_status.restype = _i
 _lib.attn_fwd_strerror.argtypes = [_i]
@@ -114,6 +119,14 @@ def attn_fwd_splitkv(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype, n_s
     return _lib.attn_fwd_splitkv(q, k, v, o, lse, B, H, Sq, Sk, D, int(causal), float(scale),
                                  int(dtype), int(n_splits), workspace, int(workspace_bytes),
                                  stream)
+
+
+def attn_fwd_splitkv_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype, n_splits,
+                             stream):
+    """The split-KV pass into the library's own per-device scratch: no workspace
+    argument, nothing allocated.  Returns the status code (no raise)."""
+    return _lib.attn_fwd_splitkv_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, int(causal),
+                                         float(scale), int(dtype), int(n_splits), stream)
 
 
 def splitkv_workspace_bytes(B, H, Sq, D, n_splits):
@@ -238,7 +251,8 @@ def attention_host(q, k, v, staging, causal=False, scale=None, out=None, lse=Non
     return out, lse
 
 
-__all__ = ["attn_fwd", "attn_fwd_host", "attn_fwd_splitkv", "attn_fwd_status", "attn_fwd_debug",
+__all__ = ["attn_fwd", "attn_fwd_host", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
+           "attn_fwd_status", "attn_fwd_debug", "SPLITKV_NOALLOC_SCRATCH_BYTES",
            "attention", "attention_splitkv", "attention_host", "splitkv_workspace_bytes",
            "splitkv_default_splits", "strerror", "abi_version", "AttnError", "ATTN_F16",
            "ATTN_BF16", "LIB_PATH", "EXPORTS"]

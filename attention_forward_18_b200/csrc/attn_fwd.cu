@@ -13,6 +13,10 @@
 #include "attn_fwd_kernel.cuh"
 #include "attn_merge.cuh"
 
+// Library-owned scratch of attn_fwd_splitkv_noalloc: one copy per device, in the
+// module's static device memory (no allocation by this library at call time).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr int kMaxSeq = 1 << 24;
@@ -85,6 +89,29 @@ int check_device(int* num_sms) {
     }
     if (num_sms) *num_sms = sms[dev];
     return verdict[dev] == 1 ? ATTN_OK : ATTN_ERR_DEVICE;
+}
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (the first lookup may load the library's device code on that device).
+int noalloc_scratch(void** out) {
+    static void* ptr[kMaxDevices];
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return ATTN_ERR_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return ATTN_ERR_LAUNCH;
+        }
+        ptr[dev] = p;
+    }
+    *out = ptr[dev];
+    return ATTN_OK;
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -351,6 +378,22 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
     if (n_splits < 1) return ATTN_ERR_SHAPE;
     return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
                reinterpret_cast<cudaStream_t>(stream), 0u, n_splits, workspace, workspace_bytes);
+}
+
+int attn_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int Sq, int Sk, int D, int causal, float scale,
+                             int dtype, int n_splits, attn_stream_t stream) {
+    int rc = validate(q, k, v, o, lse, B, H, Sq, Sk, D, scale, dtype);
+    if (rc != ATTN_OK) return rc;
+    if (n_splits < 1 || n_splits > kMaxSplits) return ATTN_ERR_SHAPE;
+    if (ws_bytes(B, H, Sq, D, n_splits) > ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES)
+        return ATTN_ERR_WORKSPACE;
+    if ((rc = check_device(nullptr)) != ATTN_OK) return rc;
+    void* scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != ATTN_OK) return rc;
+    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+               reinterpret_cast<cudaStream_t>(stream), 0u, n_splits, scratch,
+               ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES);
 }
 
 int attn_fwd_status(attn_stream_t stream, int* device_status) {

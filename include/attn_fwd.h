@@ -122,6 +122,34 @@ size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_split
  * (query block, head, range) units over the SMs best (1 .. 1024; 0 for invalid sizes). */
 int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal);
 
+/* Size of the scratch attn_fwd_splitkv_noalloc uses in place of a workspace. */
+#define ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * attn_fwd_splitkv_noalloc -- attn_fwd_splitkv for callers that must not allocate
+ * device memory for the call and cannot hand over a workspace of their own: a
+ * serving loop whose device memory is all reserved at start-up, or a plain C caller
+ * with no device allocator at hand.  The partial results go to a scratch array of
+ * ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES that the library keeps in its own static device
+ * memory, one per device; nothing is allocated per call.  (The split-KV merge is this
+ * library's; the pages have no counterpart of it or of this entry point.)
+ *   Arguments, layouts and results as attn_fwd_splitkv, without the workspace.
+ *   ATTN_ERR_WORKSPACE when attn_fwd_splitkv_workspace_bytes(B, H, Sq, D, n_splits)
+ *   exceeds ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES (use attn_fwd_splitkv, or fewer
+ *   splits); no CUDA call is made then.
+ *   The scratch needs no initialisation: every value the merge reads is written by
+ *   the same call first.
+ *   The first call on a device looks up the scratch's device address (one runtime
+ *   call, which may load the library's device code on that device) and keeps it;
+ *   make that first call before any stream capture begins.
+ *   One scratch per device: calls on one device that can overlap (different streams,
+ *   or threads without ordering) race on it and give undefined results.  Calls
+ *   ordered on one stream are safe.
+ */
+int attn_fwd_splitkv_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                             int B, int H, int Sq, int Sk, int D, int causal, float scale,
+                             int dtype, int n_splits, attn_stream_t stream);
+
 /*
  * attn_fwd_status -- synchronise `stream`, copy the current device's status word
  * into *device_status (0, or the first ATTN_ERR_* a kernel recorded since the last
