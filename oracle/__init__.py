@@ -176,5 +176,40 @@ def attn_ref_rows_ex(q, k, v, rows, mask=None, scale=1.0, causal=False, lib=None
     return o, lse
 
 
-__all__ = ["attn_ref", "attn_ref_rows", "attn_ref_ex", "attn_ref_rows_ex", "load",
+# ------------------------------------------------------------------ row softmax
+_SOFTMAX_LIB = None
+
+
+def load_softmax(path=None):
+    """Load (building first if needed) the row-softmax oracle, or the one at `path`."""
+    global _SOFTMAX_LIB
+    if path is None and _SOFTMAX_LIB is not None:
+        return _SOFTMAX_LIB
+    lib = ctypes.CDLL(path or _build.build_softmax())
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.softmax_ref_f64.argtypes = [dp, dp, ctypes.c_long, ctypes.c_long]
+    lib.softmax_ref_f64.restype = ctypes.c_int
+    lib.softmax_ref_num_threads.argtypes = []
+    lib.softmax_ref_num_threads.restype = ctypes.c_int
+    if path is None:
+        _SOFTMAX_LIB = lib
+    return lib
+
+
+def softmax_ref(x, lib=None):
+    """Row-wise softmax over the last axis of `x` (any real dtype, upcast exactly to
+    fp64): y = exp(x - max) / sum exp(x - max).  Returns fp64 of x's shape.  Follows
+    the fused-softmax paragraph of the pro.edgex.exchange summary of the tutorial."""
+    lib = lib or load_softmax()
+    x = _f64(x)
+    n = x.shape[-1] if x.ndim else 1
+    rows = x.size // n if n else 0
+    y = np.empty_like(x)
+    rc = lib.softmax_ref_f64(_ptr(x), _ptr(y), rows, n)
+    if rc != ORACLE_OK:
+        raise RuntimeError(f"oracle softmax_ref_f64 failed with code {rc}")
+    return y
+
+
+__all__ = ["softmax_ref", "load_softmax", "attn_ref", "attn_ref_rows", "attn_ref_ex", "attn_ref_rows_ex", "load",
            "num_threads", "NO_MASK", "CAUSAL_TOP_LEFT", "CAUSAL_BOTTOM_RIGHT"]

@@ -1,4 +1,5 @@
-"""Compile the fp64 CPU oracle (attn_ref.c) into oracle/liboracle_attn.so.
+"""Compile the fp64 CPU oracles: attn_ref.c into oracle/liboracle_attn.so and
+softmax_ref.c into oracle/liboracle_softmax.so.
 
 Test infrastructure only: the tests, the smoke check and the CPU-baseline leg of the
 benchmark load the result; the product path never does.
@@ -13,6 +14,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "attn_ref.c")
 LIB = os.path.join(HERE, "liboracle_attn.so")
+SOFTMAX_SRC = os.path.join(HERE, "softmax_ref.c")
+SOFTMAX_LIB = os.path.join(HERE, "liboracle_softmax.so")
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
           "-fPIC", "-shared", "-Wall", "-Wextra"]
@@ -25,11 +28,23 @@ def compile_oracle(src=SRC, out=LIB, extra=()):
     return out
 
 
+def _stale(src, lib):
+    return not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src)
+
+
 def build(force=False):
-    """Compile the oracle when the library is missing or older than its source."""
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+    """Compile the oracles when a library is missing or older than its source; returns
+    the attention oracle's path."""
+    if force or _stale(SRC, LIB):
         compile_oracle()
+    if force or _stale(SOFTMAX_SRC, SOFTMAX_LIB):
+        compile_oracle(SOFTMAX_SRC, SOFTMAX_LIB)
     return LIB
+
+
+def build_softmax(force=False):
+    build(force)
+    return SOFTMAX_LIB
 
 
 if __name__ == "__main__":
