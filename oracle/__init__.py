@@ -211,5 +211,52 @@ def softmax_ref(x, lib=None):
     return y
 
 
-__all__ = ["softmax_ref", "load_softmax", "attn_ref", "attn_ref_rows", "attn_ref_ex", "attn_ref_rows_ex", "load",
+# ------------------------------------------------------------------ GEMM + bias + act
+ACT_NONE = 0
+ACT_GELU = 1
+ACT_RELU = 2
+_GEMM_LIB = None
+
+
+def load_gemm(path=None):
+    """Load (building first if needed) the GEMM oracle, or the one at `path`."""
+    global _GEMM_LIB
+    if path is None and _GEMM_LIB is not None:
+        return _GEMM_LIB
+    lib = ctypes.CDLL(path or _build.build_gemm())
+    dp = ctypes.POINTER(ctypes.c_double)
+    lp = ctypes.c_long
+    lib.gemm_bias_act_ref_f64.argtypes = [dp, dp, dp, dp, lp, lp, lp, ctypes.c_int]
+    lib.gemm_bias_act_ref_f64.restype = ctypes.c_int
+    lib.gemm_ref_num_threads.argtypes = []
+    lib.gemm_ref_num_threads.restype = ctypes.c_int
+    if path is None:
+        _GEMM_LIB = lib
+    return lib
+
+
+def gemm_bias_act_ref(a, w, bias=None, act=ACT_NONE, lib=None):
+    """C = act(A W^T + bias) in fp64: a [M,K], w [N,K], bias [N] or None (any real
+    dtype, upcast exactly).  act: ACT_NONE, ACT_GELU (exact, erf form) or ACT_RELU.
+    Follows the GEMM-with-epilogue step of the tutorial (pro.edgex.exchange summary:
+    bias + GELU; comrad404.com summary: ReLU or bias)."""
+    lib = lib or load_gemm()
+    a, w = _f64(a), _f64(w)
+    M, K = a.shape
+    N = w.shape[0]
+    if w.shape != (N, K):
+        raise ValueError("w must be [N, K] with a's K")
+    b = _f64(bias) if bias is not None else None
+    if b is not None and b.shape != (N,):
+        raise ValueError("bias must be [N]")
+    c = np.empty((M, N), dtype=np.float64)
+    rc = lib.gemm_bias_act_ref_f64(_ptr(a), _ptr(w), _ptr(b) if b is not None else None,
+                                   _ptr(c), M, N, K, int(act))
+    if rc != ORACLE_OK:
+        raise RuntimeError(f"oracle gemm_bias_act_ref_f64 failed with code {rc}")
+    return c
+
+
+__all__ = ["gemm_bias_act_ref", "load_gemm", "ACT_NONE", "ACT_GELU", "ACT_RELU",
+           "softmax_ref", "load_softmax", "attn_ref", "attn_ref_rows", "attn_ref_ex", "attn_ref_rows_ex", "load",
            "num_threads", "NO_MASK", "CAUSAL_TOP_LEFT", "CAUSAL_BOTTOM_RIGHT"]

@@ -1,5 +1,6 @@
-"""Compile the fp64 CPU oracles: attn_ref.c into oracle/liboracle_attn.so and
-softmax_ref.c into oracle/liboracle_softmax.so.
+"""Compile the fp64 CPU oracles: attn_ref.c into oracle/liboracle_attn.so,
+softmax_ref.c into oracle/liboracle_softmax.so and gemm_ref.c into
+oracle/liboracle_gemm.so.
 
 Test infrastructure only: the tests, the smoke check and the CPU-baseline leg of the
 benchmark load the result; the product path never does.
@@ -16,6 +17,8 @@ SRC = os.path.join(HERE, "attn_ref.c")
 LIB = os.path.join(HERE, "liboracle_attn.so")
 SOFTMAX_SRC = os.path.join(HERE, "softmax_ref.c")
 SOFTMAX_LIB = os.path.join(HERE, "liboracle_softmax.so")
+GEMM_SRC = os.path.join(HERE, "gemm_ref.c")
+GEMM_LIB = os.path.join(HERE, "liboracle_gemm.so")
 
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
           "-fPIC", "-shared", "-Wall", "-Wextra"]
@@ -39,12 +42,19 @@ def build(force=False):
         compile_oracle()
     if force or _stale(SOFTMAX_SRC, SOFTMAX_LIB):
         compile_oracle(SOFTMAX_SRC, SOFTMAX_LIB)
+    if force or _stale(GEMM_SRC, GEMM_LIB):
+        compile_oracle(GEMM_SRC, GEMM_LIB)
     return LIB
 
 
 def build_softmax(force=False):
     build(force)
     return SOFTMAX_LIB
+
+
+def build_gemm(force=False):
+    build(force)
+    return GEMM_LIB
 
 
 if __name__ == "__main__":
