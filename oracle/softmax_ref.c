@@ -18,9 +18,11 @@
  * changes nothing mathematically (the factor exp(-m_r) cancels); it keeps exp from
  * overflowing.  Domain: finite inputs, n >= 1.
  *
- * Every row is checked to sum to one within 1e-12 (ORACLE_ERR_ROWSUM otherwise).
+ * Every row is checked to sum to one within 1e-12 + n * 2^-52, the rounding bound of
+ * an n-term fp64 sum (ORACLE_ERR_ROWSUM otherwise).
  * Layout: x and y rows x n, contiguous row-major fp64.  OpenMP over rows.
  */
+#include <float.h>
 #include <math.h>
 #include <stdlib.h>
 
@@ -56,7 +58,9 @@ static int softmax_one_row(const double *x, double *y, long n)
         y[j] = y[j] / l;
         total += y[j];
     }
-    return fabs(total - 1.0) <= 1e-12 ? SOFTMAX_OK : SOFTMAX_ERR_ROWSUM;
+    /* a sum of n fp64 terms of total 1 is off by at most (n - 1) * 2^-53 */
+    return fabs(total - 1.0) <= 1e-12 + (double)n * DBL_EPSILON ? SOFTMAX_OK
+                                                                 : SOFTMAX_ERR_ROWSUM;
 }
 
 int softmax_ref_f64(const double *x, double *y, long rows, long n)
