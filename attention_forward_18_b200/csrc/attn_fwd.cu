@@ -17,6 +17,9 @@
 // module's static device memory (no allocation by this library at call time).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES];
 
+// Status word of the GEMM kernels (gemm_bias_act.cu): read and cleared on `s`.
+int gemm_status_take(cudaStream_t s, int* out);
+
 namespace {
 
 constexpr int kMaxSeq = 1 << 24;
@@ -119,23 +122,27 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
+// Hkv: heads of K and V (a divisor of H; H for plain multi-head attention).
 int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
-             int B, int H, int Sq, int Sk, int D, float scale, int dtype) {
+             int B, int H, int Hkv, int Sq, int Sk, int D, float scale, int dtype) {
     if (!q || !k || !v || !o) return ATTN_ERR_NULLPTR;
     if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
     if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
-    if (B < 1 || H < 1 || Sq < 1 || Sk < 1) return ATTN_ERR_SHAPE;
+    if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || H % Hkv != 0) return ATTN_ERR_SHAPE;
     if (Sq > kMaxSeq || Sk > kMaxSeq) return ATTN_ERR_SHAPE;
     const int64_t bh = static_cast<int64_t>(B) * H;
     if (bh > kMaxHeads) return ATTN_ERR_SHAPE;
-    const int64_t n_qp = (Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
-    if (n_qp * bh > INT_MAX) return ATTN_ERR_SHAPE;
+    // the kernel's rows: g = H / Hkv query heads packed per K/V head
+    const int64_t rows = static_cast<int64_t>(H / Hkv) * Sq;
+    if (rows > kMaxSeq) return ATTN_ERR_SHAPE;
+    const int64_t n_qp = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    if (n_qp * B * Hkv > INT_MAX) return ATTN_ERR_SHAPE;
     if (!std::isfinite(scale)) return ATTN_ERR_SCALE;
     auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
     if (mis16(q) || mis16(k) || mis16(v) || mis16(o)) return ATTN_ERR_ALIGN;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return ATTN_ERR_ALIGN;
     const size_t nq = static_cast<size_t>(bh) * Sq * D * 2;
-    const size_t nk = static_cast<size_t>(bh) * Sk * D * 2;
+    const size_t nk = static_cast<size_t>(B) * Hkv * Sk * D * 2;
     if (overlaps(o, nq, q, nq) || overlaps(o, nq, k, nk) || overlaps(o, nq, v, nk))
         return ATTN_ERR_ALIAS;
     if (lse) {
@@ -147,10 +154,10 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
 }
 
-template <int D, int NS, bool BF16, bool CAUSAL, bool NEG, bool SPLIT>
+template <int D, int NS, bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
 int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const attn::Params& p, int grid, cudaStream_t stream) {
-    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG, SPLIT>;
+    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG, SPLIT, GEN>;
     constexpr int smem = attn::SmemLayout<D, NS>::ALLOC;
     static bool attr_set[kMaxDevices];
     static std::mutex mu;
@@ -176,17 +183,22 @@ template <int D>
 constexpr int kStages = (D == 64) ? 5 : 2;
 
 // Negative scales run their own instantiation (scores negated as they are read), so
-// the common case carries no per-element sign handling.
+// the common case carries no per-element sign handling.  The general causal forms
+// (an offset or grouped heads) run their own instantiations too, so plain top-left
+// causal attention keeps the simplest per-row arithmetic.
 template <int D, bool BF16, bool SPLIT>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const attn::Params& p, int grid, bool causal, cudaStream_t s) {
     const bool neg = p.scale_log2 < 0.f;
     constexpr int NS = kStages<D>;
+    if (causal && (p.causal_off != 0 || p.sq_head != p.Sq))
+        return neg ? launch_one<D, NS, BF16, true, true, SPLIT, true>(tq, tk, tv, p, grid, s)
+                   : launch_one<D, NS, BF16, true, false, SPLIT, true>(tq, tk, tv, p, grid, s);
     if (causal)
-        return neg ? launch_one<D, NS, BF16, true, true, SPLIT>(tq, tk, tv, p, grid, s)
-                   : launch_one<D, NS, BF16, true, false, SPLIT>(tq, tk, tv, p, grid, s);
-    return neg ? launch_one<D, NS, BF16, false, true, SPLIT>(tq, tk, tv, p, grid, s)
-               : launch_one<D, NS, BF16, false, false, SPLIT>(tq, tk, tv, p, grid, s);
+        return neg ? launch_one<D, NS, BF16, true, true, SPLIT, false>(tq, tk, tv, p, grid, s)
+                   : launch_one<D, NS, BF16, true, false, SPLIT, false>(tq, tk, tv, p, grid, s);
+    return neg ? launch_one<D, NS, BF16, false, true, SPLIT, false>(tq, tk, tv, p, grid, s)
+               : launch_one<D, NS, BF16, false, false, SPLIT, false>(tq, tk, tv, p, grid, s);
 }
 
 template <bool SPLIT>
@@ -225,11 +237,15 @@ int launch_merge(const float* ws_o, const float* ws_lse, void* o, float* lse, in
 
 // n_splits == 0: the whole pass (16-bit O and LSE written by the attention kernel);
 // n_splits >= 1: a split pass through `workspace`, then the merge kernel.
-int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
-        int Sk, int D, int causal, float scale, int dtype, cudaStream_t stream, unsigned flags,
-        int n_splits = 0, void* workspace = nullptr, size_t workspace_bytes = 0) {
-    int rc = validate(q, k, v, o, lse, B, H, Sq, Sk, D, scale, dtype);
+// Hkv: K/V heads (divides H); mask: ATTN_MASK_*.
+int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+        int Sq, int Sk, int D, int mask, float scale, int dtype, cudaStream_t stream,
+        unsigned flags, int n_splits = 0, void* workspace = nullptr, size_t workspace_bytes = 0) {
+    int rc = validate(q, k, v, o, lse, B, H, Hkv, Sq, Sk, D, scale, dtype);
     if (rc != ATTN_OK) return rc;
+    if (mask != ATTN_MASK_NONE && mask != ATTN_MASK_CAUSAL &&
+        mask != ATTN_MASK_CAUSAL_BOTTOM_RIGHT)
+        return ATTN_ERR_MASK;
     if (n_splits < 0 || n_splits > kMaxSplits) return ATTN_ERR_SHAPE;
     if (n_splits > 0) {
         // the merge kernel runs one warp per (head, query row) in a 1-D grid
@@ -240,7 +256,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
         const size_t need = ws_bytes(B, H, Sq, D, n_splits);
         if (workspace_bytes < need) return ATTN_ERR_WORKSPACE;
         const size_t nq = static_cast<size_t>(B) * H * Sq * D * 2;
-        const size_t nk = static_cast<size_t>(B) * H * Sk * D * 2;
+        const size_t nk = static_cast<size_t>(B) * Hkv * Sk * D * 2;
         if (overlaps(workspace, need, q, nq) || overlaps(workspace, need, k, nk) ||
             overlaps(workspace, need, v, nk) || overlaps(workspace, need, o, nq) ||
             (lse && overlaps(workspace, need, lse, static_cast<size_t>(B) * H * Sq * 4)))
@@ -249,20 +265,25 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     int num_sms = 0;
     if ((rc = check_device(&num_sms)) != ATTN_OK) return rc;
 
-    const int BH = B * H;
+    // The kernel's view: B*Hkv heads of g*Sq query rows (the g query heads of a K/V
+    // head are adjacent in [B, H, Sq, D]), Sk keys.
+    const int BH = B * Hkv;
+    const int rows = (H / Hkv) * Sq;
     const bool bf16 = dtype == ATTN_BF16;
     CUtensorMap tq, tk, tv;
-    if (!encode_qkv_map(&tq, q, D, Sq, BH, bf16) || !encode_qkv_map(&tk, k, D, Sk, BH, bf16) ||
+    if (!encode_qkv_map(&tq, q, D, rows, BH, bf16) || !encode_qkv_map(&tk, k, D, Sk, BH, bf16) ||
         !encode_qkv_map(&tv, v, D, Sk, BH, bf16))
         return ATTN_ERR_TENSORMAP;
 
     attn::Params p;
     p.o = o;
     p.lse = lse;
-    p.Sq = Sq;
+    p.Sq = rows;
     p.Sk = Sk;
     p.BH = BH;
-    p.n_qp = (Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    p.n_qp = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    p.sq_head = Sq;
+    p.causal_off = mask == ATTN_MASK_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
     const int n_kv = (Sk + attn::BN - 1) / attn::BN;
     p.n_splits = n_splits > 0 ? n_splits : 1;
     p.chunk_tiles = (n_kv + p.n_splits - 1) / p.n_splits;
@@ -280,12 +301,37 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int64_t n_units = static_cast<int64_t>(p.n_qp) * BH * p.n_splits;
     if (n_units > INT_MAX) return ATTN_ERR_SHAPE;
     const int grid = n_units < num_sms ? static_cast<int>(n_units) : num_sms;
-    const bool c = causal != 0;
+    const bool c = mask != ATTN_MASK_NONE;
     if (n_splits == 0) return launch_any<false>(tq, tk, tv, p, grid, D, bf16, c, stream);
     rc = launch_any<true>(tq, tk, tv, p, grid, D, bf16, c, stream);
     if (rc != ATTN_OK) return rc;
-    return launch_merge(p.ws_o, p.ws_lse, o, lse, n_splits, static_cast<int64_t>(BH) * Sq, D,
+    return launch_merge(p.ws_o, p.ws_lse, o, lse, n_splits, static_cast<int64_t>(B) * H * Sq, D,
                         bf16, stream);
+}
+
+int mask_of(int causal) { return causal ? ATTN_MASK_CAUSAL : ATTN_MASK_NONE; }
+
+// Split count for `units` (query block, head) pairs over KV tiles 0..n_kv-1: persistent
+// CTAs take units round-robin, so a pass lasts about
+//   ceil(units * n / SMs) rounds x (tiles per range + a fill of ~2 tiles);
+// the n with the least of that (the fewest splits among equals: less to merge).
+int balanced_splits(int64_t units, int n_kv) {
+    int num_sms = 0;
+    if (check_device(&num_sms) != ATTN_OK) num_sms = 148;
+    int best = 1;
+    int64_t best_cost = INT64_MAX;
+    const int n_hi = n_kv < kMaxSplits ? n_kv : kMaxSplits;
+    for (int n = 1; n <= n_hi; ++n) {
+        const int chunk = (n_kv + n - 1) / n;
+        if ((n_kv + chunk - 1) / chunk != n) continue;  // some range would be empty
+        const int64_t rounds = (units * n + num_sms - 1) / num_sms;
+        const int64_t cost = rounds * (chunk + 2);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = n;
+        }
+    }
+    return best;
 }
 
 }  // namespace
@@ -294,14 +340,14 @@ extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int Sq, int Sk, int D, int causal, float scale, int dtype, attn_stream_t stream) {
-    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+    return run(q, k, v, o, lse, B, H, H, Sq, Sk, D, mask_of(causal), scale, dtype,
                reinterpret_cast<cudaStream_t>(stream), 0u);
 }
 
 int attn_fwd_debug(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                    int H, int Sq, int Sk, int D, int causal, float scale, int dtype,
                    attn_stream_t stream, unsigned flags) {
-    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+    return run(q, k, v, o, lse, B, H, H, Sq, Sk, D, mask_of(causal), scale, dtype,
                reinterpret_cast<cudaStream_t>(stream), flags & attn::FLAG_SKIP_Q_LOAD);
 }
 
@@ -310,7 +356,7 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
                   float* lse_dev, int B, int H, int Sq, int Sk, int D, int causal, float scale,
                   int dtype, attn_stream_t stream) {
     if (!q_host || !k_host || !v_host || !o_host) return ATTN_ERR_NULLPTR;
-    int rc = validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Sq, Sk, D, scale, dtype);
+    int rc = validate(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, H, Sq, Sk, D, scale, dtype);
     if (rc != ATTN_OK) return rc;
     if ((rc = check_device(nullptr)) != ATTN_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -322,7 +368,8 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }
-    rc = run(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Sq, Sk, D, causal, scale, dtype, s, 0u);
+    rc = run(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, H, Sq, Sk, D, mask_of(causal), scale,
+             dtype, s, 0u);
     if (rc != ATTN_OK) return rc;
     if (cudaMemcpyAsync(o_host, o_dev, nq, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
         cudaGetLastError();
@@ -344,31 +391,18 @@ size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_split
 }
 
 int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal) {
-    if (B < 1 || H < 1 || Sq < 1 || Sk < 1) return 0;
-    int num_sms = 0;
-    if (check_device(&num_sms) != ATTN_OK) num_sms = 148;
-    const int64_t units = static_cast<int64_t>((Sq + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA) *
-                          B * H;
+    return attn_fwd_ex_default_splits(B, H, H, Sq, Sk, mask_of(causal));
+}
+
+int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int mask) {
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Sq < 1 || Sk < 1 || mask < 0 ||
+        mask > ATTN_MASK_CAUSAL_BOTTOM_RIGHT)
+        return 0;
+    const int64_t rows = static_cast<int64_t>(H / H_kv) * Sq;
+    const int64_t units = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA * B * H_kv;
     // with the top-left causal mask no row sees a key past min(Sq, Sk)
-    const int keys = causal ? (Sq < Sk ? Sq : Sk) : Sk;
-    const int n_kv = (keys + attn::BN - 1) / attn::BN;
-    // Persistent CTAs take units round-robin, so the pass lasts about
-    //   ceil(units * n / SMs) rounds x (tiles per range + a fill of ~2 tiles);
-    // take the n with the least of that (the fewest splits among equals: less to merge).
-    int best = 1;
-    int64_t best_cost = INT64_MAX;
-    const int n_hi = n_kv < kMaxSplits ? n_kv : kMaxSplits;
-    for (int n = 1; n <= n_hi; ++n) {
-        const int chunk = (n_kv + n - 1) / n;
-        if ((n_kv + chunk - 1) / chunk != n) continue;  // some range would be empty
-        const int64_t rounds = (units * n + num_sms - 1) / num_sms;
-        const int64_t cost = rounds * (chunk + 2);
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = n;
-        }
-    }
-    return best;
+    const int keys = mask == ATTN_MASK_CAUSAL ? (Sq < Sk ? Sq : Sk) : Sk;
+    return balanced_splits(units, (keys + attn::BN - 1) / attn::BN);
 }
 
 int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -376,14 +410,21 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
                      int n_splits, void* workspace, size_t workspace_bytes,
                      attn_stream_t stream) {
     if (n_splits < 1) return ATTN_ERR_SHAPE;
-    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+    return run(q, k, v, o, lse, B, H, H, Sq, Sk, D, mask_of(causal), scale, dtype,
+               reinterpret_cast<cudaStream_t>(stream), 0u, n_splits, workspace, workspace_bytes);
+}
+
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int H_kv, int Sq, int Sk, int D, int mask, float scale, int dtype, int n_splits,
+                void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    return run(q, k, v, o, lse, B, H, H_kv, Sq, Sk, D, mask, scale, dtype,
                reinterpret_cast<cudaStream_t>(stream), 0u, n_splits, workspace, workspace_bytes);
 }
 
 int attn_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int H, int Sq, int Sk, int D, int causal, float scale,
                              int dtype, int n_splits, attn_stream_t stream) {
-    int rc = validate(q, k, v, o, lse, B, H, Sq, Sk, D, scale, dtype);
+    int rc = validate(q, k, v, o, lse, B, H, H, Sq, Sk, D, scale, dtype);
     if (rc != ATTN_OK) return rc;
     if (n_splits < 1 || n_splits > kMaxSplits) return ATTN_ERR_SHAPE;
     if (ws_bytes(B, H, Sq, D, n_splits) > ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES)
@@ -391,7 +432,7 @@ int attn_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* 
     if ((rc = check_device(nullptr)) != ATTN_OK) return rc;
     void* scratch = nullptr;
     if ((rc = noalloc_scratch(&scratch)) != ATTN_OK) return rc;
-    return run(q, k, v, o, lse, B, H, Sq, Sk, D, causal, scale, dtype,
+    return run(q, k, v, o, lse, B, H, H, Sq, Sk, D, mask_of(causal), scale, dtype,
                reinterpret_cast<cudaStream_t>(stream), 0u, n_splits, scratch,
                ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES);
 }
@@ -410,7 +451,10 @@ int attn_fwd_status(attn_stream_t stream, int* device_status) {
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }
-    *device_status = value;
+    // the GEMM kernels keep their own word (another translation unit)
+    int gemm_value = 0;
+    if (gemm_status_take(s, &gemm_value) != ATTN_OK) return ATTN_ERR_LAUNCH;
+    *device_status = value != 0 ? value : gemm_value;
     return ATTN_OK;
 }
 
@@ -428,6 +472,7 @@ const char* attn_fwd_strerror(int code) {
         case ATTN_ERR_SCALE: return "scale is not finite";
         case ATTN_ERR_ALIAS: return "output overlaps an input";
         case ATTN_ERR_DEVICE: return "no usable sm_100 CUDA device";
+        case ATTN_ERR_MASK: return "mask is not one of ATTN_MASK_*";
         case ATTN_ERR_WORKSPACE: return "workspace smaller than attn_fwd_splitkv_workspace_bytes";
         default: return "unknown error code";
     }

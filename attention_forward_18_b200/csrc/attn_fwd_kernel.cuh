@@ -73,12 +73,18 @@ constexpr int STATUS_TIMEOUT = -8;  // ATTN_ERR_TIMEOUT
 // out; only the timeout test sets it.
 constexpr uint32_t FLAG_SKIP_Q_LOAD = 1u;
 
+// Rows and heads as the kernel sees them: with grouped K/V heads (g query heads per
+// K/V head) the g query heads of a group are adjacent in [B, H, Sq, D], so Q, O and
+// LSE are read as [B*Hkv, g*Sq, ...] and one "head" of the kernel is a K/V head with
+// g*Sq query rows; packed row r is query position r % sq_head.
 struct Params {
     void* o;            // [BH, Sq, D] 16-bit (whole pass)
     float* lse;         // [BH, Sq] fp32, may be null (whole pass)
     float* ws_o;        // split-KV: [n_splits, BH, Sq, D] fp32 partial O (normalised)
     float* ws_lse;      // split-KV: [n_splits, BH, Sq] fp32 partial LSE
-    int Sq, Sk, BH, n_qp;
+    int Sq, Sk, BH, n_qp;  // packed query rows, keys, K/V heads, 256-row query pairs
+    int sq_head;        // query positions per query head (Sq / g)
+    int causal_off;     // causal: key j visible to position i iff j <= i + causal_off
     int n_splits;       // KV ranges per (query pair, head); 1 for the whole pass
     int chunk_tiles;    // KV tiles per range
     float scale_log2;   // scale * log2(e)
@@ -167,7 +173,23 @@ struct Unit {
     int n[2];
 };
 
-template <bool CAUSAL, bool SPLIT>
+// Causal visibility bound of packed rows first..last: the last key visible to the
+// row at the largest query position (LEAST = false) or to the row at the smallest one
+// (LEAST = true).  The rows span a head boundary only with grouped heads.
+template <bool LEAST>
+__device__ __forceinline__ int tile_vis(int first, int last, const Params& p) {
+    int pos;
+    if (p.sq_head == p.Sq) {
+        pos = LEAST ? first : last;
+    } else if (first / p.sq_head != last / p.sq_head) {
+        pos = LEAST ? 0 : p.sq_head - 1;
+    } else {
+        pos = (LEAST ? first : last) % p.sq_head;
+    }
+    return pos + p.causal_off;
+}
+
+template <bool CAUSAL, bool SPLIT, bool GEN>
 __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     Unit w;
     w.split = SPLIT ? u % p.n_splits : 0;
@@ -186,7 +208,12 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     for (int t = 0; t < 2; ++t) {
         const int first = w.qp * ROWS_PER_CTA + BM * t;
         int end = kv_end;
-        if (CAUSAL) end = min(end, (min(first + BM - 1, p.Sq - 1)) / BN + 1);
+        if (CAUSAL) {
+            // the last key any row of the tile sees
+            const int last = min(first + BM - 1, p.Sq - 1);
+            const int vis = GEN ? tile_vis<false>(first, last, p) : last;
+            end = vis < 0 ? 0 : min(end, vis / BN + 1);
+        }
         w.n[t] = (first >= p.Sq) ? 0 : max(0, end - w.kv0);
     }
     return w;
@@ -229,7 +256,7 @@ __device__ __forceinline__ void scores_ready(uint32_t (&s)[128], int half) {
 // every visible p is then 2^(~1e-28) = 1.0f exactly, the uniform weights a zero
 // scale gives, and masked scores stay -inf).  Returns alpha, the factor O must be
 // scaled by before P_j V_j is added (1 = none).
-template <bool IS_BF16, bool NEG, bool MASK>
+template <bool IS_BF16, bool NEG, bool MASK, bool GEN>
 __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, float c,
                                                    float& m_used, float& l) {
     uint32_t s[128];
@@ -256,7 +283,7 @@ __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, 
     max64(&s[64], a);
     const float mx =
         ptx::max3(ptx::max3(a[0], a[1], a[2]), ptx::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-    // every processed tile has a visible key in every row, so mx is finite here
+    // mx = -inf only for a row that sees no key of this (masked) tile
     const float m_tile = mx * c;
     float alpha = 1.f;
     if (j == 0) {
@@ -265,7 +292,9 @@ __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, 
         alpha = ptx::ex2(m_used - m_tile);
         m_used = m_tile;
     }
-    const float neg_m = -m_used;
+    // a row that has seen no key yet keeps m = -inf (possible only in a masked tile of
+    // the general causal forms: bottom-right offsets, grouped heads); its p must be 0
+    const float neg_m = (MASK && GEN && m_used == -INFINITY) ? 0.f : -m_used;
 
     // p = 2^(s * c - m): scale and shift in one packed fma per column pair; the row
     // sum accumulates in a packed pair too
@@ -292,17 +321,20 @@ __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, 
 }
 
 // The tile's masking is decided once, by a warp-uniform branch, so the unmasked tiles
-// (all but the last and, causally, the diagonal one) run the loops without it.
-template <bool IS_BF16, bool CAUSAL, bool NEG>
-__device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int qrow,
-                                              int q0t, float c, float& m_used, float& l) {
-    const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > q0t);
+// (all but the last and, causally, the diagonal ones) run the loops without it.
+// row_vis: the last key this row sees; tile_vis_min: the least of that over the
+// tile's rows (causal only).
+template <bool IS_BF16, bool CAUSAL, bool NEG, bool GEN>
+__device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int row_vis,
+                                              int tile_vis_min, float c, float& m_used,
+                                              float& l) {
+    const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > tile_vis_min);
     if (need_mask) {
         int lim = Sk - 1 - kv0;
-        if (CAUSAL) lim = min(lim, qrow - kv0);
-        return softmax_tile_body<IS_BF16, NEG, true>(tS, j, lim, c, m_used, l);
+        if (CAUSAL) lim = min(lim, row_vis - kv0);
+        return softmax_tile_body<IS_BF16, NEG, true, GEN>(tS, j, lim, c, m_used, l);
     }
-    return softmax_tile_body<IS_BF16, NEG, false>(tS, j, 0, c, m_used, l);
+    return softmax_tile_body<IS_BF16, NEG, false, GEN>(tS, j, 0, c, m_used, l);
 }
 
 // The r-th unit of this CTA in a boustrophedon order over the grid (round r takes
@@ -315,7 +347,10 @@ __device__ __forceinline__ int unit_of(int r, int n_units) {
     return u < n_units ? u : -1;
 }
 
-template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT>
+// GEN (causal only): the general causal forms -- a nonzero offset (bottom-right
+// alignment) or grouped query heads packed into one sequence; without it a row's
+// position is its row index and the offset is 0, and no row is ever fully masked.
+template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -407,16 +442,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int u = unit_of(r, n_units);
             if (u < 0) break;
-            const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
+            const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
             const int q0t = w.qp * ROWS_PER_CTA + BM * t;
             const int qrow = q0t + row;
             const int n_t = w.n[t];
+            int row_vis = qrow, tile_vis_min = q0t;
+            if (GEN && n_t > 0) {
+                row_vis = (p.sq_head == p.Sq ? qrow : qrow % p.sq_head) + p.causal_off;
+                tile_vis_min = tile_vis<true>(q0t, min(q0t + BM - 1, p.Sq - 1), p);
+            }
             float m_used = -INFINITY, l = 0.f;
             for (int j = 0; j < n_t; ++j, ++it) {
                 if (!(ok = warp_wait(ctx, B_SF(t), it & 1))) break;
                 ptx::tc_fence_after();
-                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG>(
-                    tS, j, (w.kv0 + j) * BN, p.Sk, qrow, q0t, c_abs, m_used, l);
+                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG, GEN>(
+                    tS, j, (w.kv0 + j) * BN, p.Sk, row_vis, tile_vis_min, c_abs, m_used, l);
                 // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
                 // bring it to the new max before PV_t,j adds to it
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -457,18 +497,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int r = 0; ok; ++r) {
             const int u = unit_of(r, n_units);
             if (u < 0) break;
-            const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
+            const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
             const int64_t head_row = static_cast<int64_t>(w.split) * p.BH + w.bh;
             for (int t = 0; ok && t < 2; ++t) {
                 const int qrow = w.qp * ROWS_PER_CTA + BM * t + row;
                 const bool store = qrow < p.Sq;
                 if (w.n[t] == 0) {
-                    // split pass: no key of this range is visible to these rows
+                    // no key of the unit's range is visible to these rows: O = 0 and
+                    // LSE = -inf (the empty sum)
                     if (SPLIT && store) {
                         float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D);
 #pragma unroll 1
                         for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
                         p.ws_lse[head_row * p.Sq + qrow] = -INFINITY;
+                    } else if (!SPLIT && store) {
+                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                                              (static_cast<int64_t>(w.bh) * p.Sq + qrow) * D);
+#pragma unroll 1
+                        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+                        if (p.lse != nullptr) p.lse[static_cast<int64_t>(w.bh) * p.Sq + qrow] = -INFINITY;
                     }
                     continue;
                 }
@@ -593,7 +640,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
-                    const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
+                    const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
                     const int n_t[2] = {w.n[0], w.n[1]};
                     const int n_max = max(n_t[0], n_t[1]);
                     if (n_max == 0) continue;  // a split range no query row of the unit sees
@@ -653,7 +700,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
-                    const Unit w = decode_unit<CAUSAL, SPLIT>(u, p);
+                    const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
                     const int q0 = w.qp * ROWS_PER_CTA;
                     const int bh = w.bh;
                     const int n_max = max(w.n[0], w.n[1]);

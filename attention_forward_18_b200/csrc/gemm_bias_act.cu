@@ -1,0 +1,460 @@
+// gemm_bias_act.cu -- C = act(A W^T + bias) on the sm_100a tensor cores, the C ABI of
+// include/gemm_bias_act.h.
+//
+// Persistent, warp-specialised, one CTA per SM (384 threads):
+//   warp 0       TMA producer: 128x64 tiles of A and 256x64 tiles of W (128-byte
+//                swizzle) into a 4-stage shared-memory ring (48 KB per stage);
+//   warp 1       MMA issuer: per 64-wide K block four tcgen05.mma (M=128, N=256,
+//                K=16) into one of two fp32 accumulators in tensor memory (2 x 256
+//                columns), so the epilogue of one tile overlaps the products of the
+//                next;
+//   warp 2       tensor-memory allocation / release;
+//   warps 4..11  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lane
+//                quarter w % 4, column half (w - 4) / 4), + bias, activation in fp32,
+//                one rounding to 16 bits, 16-byte stores.
+// Output tiles are visited in groups of 8 M-blocks (N-blocks inner within a group) so
+// the CTAs running at one time share their A and W tiles in L2.
+// Every wait is bounded (2 s); a timeout records ATTN_ERR_TIMEOUT in this file's
+// status word (read through attn_fwd_status), all roles leave their loops, in-flight
+// copies and MMAs are drained (bounded) and tensor memory is freed.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include "attn_fwd.h"
+#include "gemm_bias_act.h"
+#include "ptx.cuh"
+
+namespace gemm {
+
+namespace ptx = attn::ptx;
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;           // 16 KB
+constexpr int B_BYTES = BN * BK * 2;           // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
+constexpr int NUM_THREADS = 384;
+constexpr int EPI_WARP0 = 4, EPI_WARPS = 8;
+constexpr int GROUP_M = 8;
+constexpr uint32_t TMEM_COLS = 512;            // two 256-column accumulators
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;
+constexpr int STATUS_TIMEOUT = -8;             // ATTN_ERR_TIMEOUT
+
+// shared memory: ring | barriers | tmem slot, error flag
+constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+// full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+constexpr int NBAR = 2 * STAGES + 5;
+constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
+static_assert(2 * SMEM_BYTES > 232448, "one CTA per SM (it takes all of TMEM)");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct Params {
+    void* c;              // [M, N] 16-bit
+    const void* bias;     // [N] 16-bit or null
+    int M, N, K;
+    int num_m, num_n, num_k, num_tiles;
+    uint32_t flags;       // bit 0: the producer skips its loads (timeout test)
+};
+
+__device__ int g_gemm_status;
+
+struct Ctx {
+    volatile int* err;
+};
+
+__device__ __forceinline__ void raise_error(const Ctx& c, int code) {
+    *c.err = 1;
+    atomicCAS(&g_gemm_status, 0, code);
+}
+
+__device__ __forceinline__ bool wait_bounded(const Ctx& c, uint32_t bar, uint32_t parity) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*c.err) return false;
+        if (ptx::globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            raise_error(c, STATUS_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer_ns() - t0 > DRAIN_LIMIT_NS) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool warp_wait(const Ctx& c, uint32_t bar, uint32_t parity) {
+    const bool ok = wait_bounded(c, bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Output tile t -> (M-block, N-block): groups of GROUP_M M-blocks, N-blocks outer
+// within a group.
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
+    const int per_group = GROUP_M * p.num_n;
+    const int g = t / per_group;
+    const int first = g * GROUP_M;
+    const int rows = min(p.num_m - first, GROUP_M);
+    const int r = t - g * per_group;
+    mb = first + r % rows;
+    nb = r / rows;
+}
+
+template <int ACT>
+__device__ __forceinline__ float activate(float z) {
+    if constexpr (ACT == GEMM_ACT_GELU) return 0.5f * z * (1.f + erff(z * 0.70710678118654752f));
+    else if constexpr (ACT == GEMM_ACT_RELU) return fmaxf(z, 0.f);
+    else return z;
+}
+
+template <bool IS_BF16>
+__device__ __forceinline__ float load16(const void* p, int i) {
+    const uint16_t b = reinterpret_cast<const uint16_t*>(p)[i];
+    if constexpr (IS_BF16) return __uint_as_float(static_cast<uint32_t>(b) << 16);
+    else return __half2float(__ushort_as_half(b));
+}
+
+template <bool IS_BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    if constexpr (IS_BF16) return ptx::pack_bf16x2(lo, hi);
+    else return ptx::pack_f16x2(lo, hi);
+}
+
+template <bool IS_BF16, int ACT, bool HAS_BIAS>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_bias_act_kernel(const __grid_constant__ CUtensorMap tm_a,
+                         const __grid_constant__ CUtensorMap tm_w, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = ptx::smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const uint32_t bars = sbase + BAR_OFF;
+    auto B_FULL = [&](int s) { return bars + 8u * s; };
+    auto B_EMPTY = [&](int s) { return bars + 8u * (STAGES + s); };
+    auto B_AF = [&](int b) { return bars + 8u * (2 * STAGES + b); };      // accumulator b done
+    auto B_AE = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };  // accumulator b read
+    const uint32_t B_DR = bars + 8u * (2 * STAGES + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + MISC_OFF);
+    Ctx ctx{reinterpret_cast<volatile int*>(smem + MISC_OFF + 4)};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(B_FULL(s), 1);
+            ptx::mbar_init(B_EMPTY(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(B_AF(b), 1);
+            ptx::mbar_init(B_AE(b), EPI_WARPS);
+        }
+        ptx::mbar_init(B_DR, 1);
+        *ctx.err = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================================ TMA producer
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_a);
+            ptx::prefetch_tmap(&tm_w);
+            const bool load = !(p.flags & 1u);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+                int mb, nb;
+                tile_coords(t, p, mb, nb);
+                for (int kb = 0; kb < p.num_k; ++kb, ++it) {
+                    const int s = static_cast<int>(it % STAGES);
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!(ok = wait_bounded(ctx, B_EMPTY(s), ph ^ 1u))) break;
+                    if (!load) continue;
+                    const uint32_t sa = sbase + s * STAGE_BYTES;
+                    ptx::mbar_arrive_expect_tx(B_FULL(s), STAGE_BYTES);
+                    ptx::tma_load_2d(sa, &tm_a, B_FULL(s), kb * BK, mb * BM);
+                    ptx::tma_load_2d(sa + A_BYTES, &tm_w, B_FULL(s), kb * BK, nb * BN);
+                }
+            }
+            // let the copies in flight land before the CTA can exit
+            if (load) {
+                const uint32_t n = it < STAGES ? it : STAGES;
+                for (uint32_t q = it - n; q < it; ++q)
+                    wait_drain(B_FULL(static_cast<int>(q % STAGES)), (q / STAGES) & 1u);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::idesc_f16(IS_BF16 ? 1u : 0u, BM, BN, 0);
+            constexpr uint32_t hi = ptx::smem_desc_hi_sw128(1024);
+            uint32_t it = 0, i = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++i) {
+                const int ab = static_cast<int>(i & 1u);
+                if (!(ok = wait_bounded(ctx, B_AE(ab), ((i >> 1) & 1u) ^ 1u))) break;
+                ptx::tc_fence_after();
+                const uint32_t d = tmem + static_cast<uint32_t>(ab) * BN;
+                for (int kb = 0; kb < p.num_k; ++kb, ++it) {
+                    const int s = static_cast<int>(it % STAGES);
+                    if (!(ok = wait_bounded(ctx, B_FULL(s), (it / STAGES) & 1u))) break;
+                    ptx::tc_fence_after();
+                    const uint32_t sa = sbase + s * STAGE_BYTES;
+                    const uint32_t a_lo = ptx::smem_desc_lo(sa, 16);
+                    const uint32_t b_lo = ptx::smem_desc_lo(sa + A_BYTES, 16);
+                    // K steps of 16 elements: +32 bytes inside the 128-byte swizzled row
+                    ptx::mma_ss_off<0, 0>(d, a_lo, b_lo, hi, idesc, kb > 0 ? 1u : 0u);
+                    ptx::mma_ss_off<2, 2>(d, a_lo, b_lo, hi, idesc, 1u);
+                    ptx::mma_ss_off<4, 4>(d, a_lo, b_lo, hi, idesc, 1u);
+                    ptx::mma_ss_off<6, 6>(d, a_lo, b_lo, hi, idesc, 1u);
+                    ptx::mma_commit(B_EMPTY(s));
+                }
+                if (!ok) break;
+                ptx::mma_commit(B_AF(ab));
+            }
+            // every MMA issued above completes before tensor memory is freed
+            ptx::mma_commit(B_DR);
+            wait_drain(B_DR, 0);
+        }
+        __syncwarp();
+    } else if (warp >= EPI_WARP0) {
+        // ================================================================ epilogue
+        const int q = warp & 3;                   // TMEM lane quarter
+        const int half = (warp - EPI_WARP0) >> 2;  // column half of the tile
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        uint32_t i = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++i) {
+            int mb, nb;
+            tile_coords(t, p, mb, nb);
+            const int ab = static_cast<int>(i & 1u);
+            if (!(ok = warp_wait(ctx, B_AF(ab), (i >> 1) & 1u))) break;
+            ptx::tc_fence_after();
+            const int row = mb * BM + q * 32 + lane;
+            const bool row_ok = row < p.M;
+            uint16_t* crow = reinterpret_cast<uint16_t*>(p.c) + static_cast<int64_t>(row) * p.N;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                const int col0 = nb * BN + half * 128 + c * 32;
+                uint32_t v[32];
+                ptx::tmem_ld32(tmem + lane_base + static_cast<uint32_t>(ab * BN + half * 128 + c * 32), v);
+                ptx::tmem_wait_ld();
+                ptx::reg_fence32(v);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int cg = col0 + 8 * g;  // N is a multiple of 8: groups are whole
+                    if (cg >= p.N) continue;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float z0 = __uint_as_float(v[8 * g + 2 * e]);
+                        float z1 = __uint_as_float(v[8 * g + 2 * e + 1]);
+                        if constexpr (HAS_BIAS) {
+                            z0 += load16<IS_BF16>(p.bias, cg + 2 * e);
+                            z1 += load16<IS_BF16>(p.bias, cg + 2 * e + 1);
+                        }
+                        w[e] = pack2<IS_BF16>(activate<ACT>(z0), activate<ACT>(z1));
+                    }
+                    if (row_ok)
+                        *reinterpret_cast<uint4*>(crow + cg) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            // the accumulator is read: the MMA warp may start the tile after next in it
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(B_AE(ab));
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace gemm
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [rows, K] 16-bit row-major as a 2-D tensor (K innermost); box 64 x box_rows with
+// the 128-byte swizzle; out-of-range rows / columns read as zeros.
+bool encode_2d(CUtensorMap* m, const void* base, int K, int rows, int box_rows, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm::BK),
+                               static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sms() {
+    static int sms[64];
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return -1;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (sms[dev] == 0) {
+        int major = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return -1;
+        }
+        sms[dev] = (major == 10 && n > 0) ? n : -1;
+    }
+    return sms[dev];
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+template <bool BF16, int ACT, bool BIAS>
+int launch(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p, int grid,
+           cudaStream_t s) {
+    auto k = gemm::gemm_bias_act_kernel<BF16, ACT, BIAS>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    k<<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, s>>>(ta, tw, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <bool BF16, int ACT>
+int launch_bias(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p, int grid,
+                cudaStream_t s) {
+    return p.bias ? launch<BF16, ACT, true>(ta, tw, p, grid, s)
+                  : launch<BF16, ACT, false>(ta, tw, p, grid, s);
+}
+
+template <bool BF16>
+int launch_act(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p, int act,
+               int grid, cudaStream_t s) {
+    if (act == GEMM_ACT_GELU) return launch_bias<BF16, GEMM_ACT_GELU>(ta, tw, p, grid, s);
+    if (act == GEMM_ACT_RELU) return launch_bias<BF16, GEMM_ACT_RELU>(ta, tw, p, grid, s);
+    return launch_bias<BF16, GEMM_ACT_NONE>(ta, tw, p, grid, s);
+}
+
+int run(const void* a, const void* w, const void* bias, void* c, int M, int N, int K, int act,
+        int dtype, cudaStream_t stream, unsigned flags) {
+    if (!a || !w || !c) return ATTN_ERR_NULLPTR;
+    if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
+    if (act != GEMM_ACT_NONE && act != GEMM_ACT_GELU && act != GEMM_ACT_RELU) return ATTN_ERR_SHAPE;
+    if (M < 1 || N < 1 || K < 1 || N % 8 != 0 || K % 8 != 0) return ATTN_ERR_SHAPE;
+    auto mis16 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) != 0; };
+    if (mis16(a) || mis16(w) || mis16(c)) return ATTN_ERR_ALIGN;
+    if (bias && (reinterpret_cast<uintptr_t>(bias) & 1u)) return ATTN_ERR_ALIGN;
+    const size_t na = static_cast<size_t>(M) * K * 2, nw = static_cast<size_t>(N) * K * 2;
+    const size_t nc = static_cast<size_t>(M) * N * 2;
+    if (overlaps(c, nc, a, na) || overlaps(c, nc, w, nw) ||
+        (bias && overlaps(c, nc, bias, static_cast<size_t>(N) * 2)))
+        return ATTN_ERR_ALIAS;
+    const int sms = device_sms();
+    if (sms < 1) return ATTN_ERR_DEVICE;
+    const bool bf16 = dtype == ATTN_BF16;
+    CUtensorMap ta, tw;
+    if (!encode_2d(&ta, a, K, M, gemm::BM, bf16) || !encode_2d(&tw, w, K, N, gemm::BN, bf16))
+        return ATTN_ERR_TENSORMAP;
+    gemm::Params p;
+    p.c = c;
+    p.bias = bias;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.num_m = (M + gemm::BM - 1) / gemm::BM;
+    p.num_n = (N + gemm::BN - 1) / gemm::BN;
+    p.num_k = (K + gemm::BK - 1) / gemm::BK;
+    const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
+    if (tiles > INT_MAX) return ATTN_ERR_SHAPE;
+    p.num_tiles = static_cast<int>(tiles);
+    p.flags = flags;
+    const int grid = p.num_tiles < sms ? p.num_tiles : sms;
+    return bf16 ? launch_act<true>(ta, tw, p, act, grid, stream)
+                : launch_act<false>(ta, tw, p, act, grid, stream);
+}
+
+}  // namespace
+
+// Read and clear this file's status word (attn_fwd_status reports it with the
+// attention kernels' word).  Internal to the library.
+__attribute__((visibility("hidden"))) int gemm_status_take(cudaStream_t s, int* out) {
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, gemm::g_gemm_status, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(gemm::g_gemm_status, &zero, sizeof(int), 0,
+                                cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_LAUNCH;
+    }
+    *out = v;
+    return ATTN_OK;
+}
+
+extern "C" {
+
+int gemm_bias_act(const void* a, const void* w, const void* bias, void* c, int M, int N, int K,
+                  int act, int dtype, attn_stream_t stream) {
+    return run(a, w, bias, c, M, N, K, act, dtype, reinterpret_cast<cudaStream_t>(stream), 0u);
+}
+
+int gemm_bias_act_debug(const void* a, const void* w, const void* bias, void* c, int M, int N,
+                        int K, int act, int dtype, attn_stream_t stream, unsigned flags) {
+    return run(a, w, bias, c, M, N, K, act, dtype, reinterpret_cast<cudaStream_t>(stream),
+               flags & 1u);
+}
+
+}  // extern "C"

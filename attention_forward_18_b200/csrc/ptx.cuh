@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the attention
-// kernel uses: mbarriers, TMA tensor loads, tensor memory (TMEM) allocation and
+// and GEMM kernels use: mbarriers, TMA tensor loads, tensor memory (TMEM) allocation and
 // access, and tcgen05 MMAs.  Each wrapper is one PTX instruction (or a fixed
 // handful), written from the PTX ISA's description of that instruction.
 #pragma once
@@ -71,6 +71,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+
+// 2-D tiled tensor load global -> shared (same rules: c0 innermost, a multiple of
+// 8 elements for 16-bit data; the out-of-range part of the box reads as zeros).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint32_t bar,
+                                            int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
 

@@ -62,6 +62,9 @@ def parse():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--profile-once", action="store_true",
                     help="launch each pass of the workload once and exit (for ncu captures)")
+    ap.add_argument("--profile-extra", default=None,
+                    help="with --profile-once: a DEC*, SMX* or GEMM* workload instead, optionally "
+                         "scaled down as NAME:rows (M for GEMM*, rows for SMX*, B for DEC*)")
     return ap.parse_args()
 
 
@@ -394,26 +397,27 @@ def decode_workloads(names):
         o = torch.empty_like(q)
         lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
         dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
-        n = af.splitkv_default_splits(w.B, w.H, w.Sq, w.Sk, False)
+        Hkv = w.kv_heads
+        n = af.ex_default_splits(w.B, w.H, Hkv, w.Sq, w.Sk, af.ATTN_MASK_NONE)
         nbytes = af.splitkv_workspace_bytes(w.B, w.H, w.Sq, w.D, n)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                w.B, w.H, w.Sq, w.Sk, w.D, 0, w.scale, dcode)
+                w.B, w.H, Hkv, w.Sq, w.Sk, w.D, af.ATTN_MASK_NONE, w.scale, dcode)
 
         def split():
-            rc = af.attn_fwd_splitkv(*args, n, ws.data_ptr(), nbytes, stream.cuda_stream)
+            rc = af.attn_fwd_ex(*args, n, ws.data_ptr(), nbytes, stream.cuda_stream)
             if rc != 0:
-                raise af.AttnError(rc, "attn_fwd_splitkv")
+                raise af.AttnError(rc, "attn_fwd_ex")
 
         def whole():
-            rc = af.attn_fwd(*args, stream.cuda_stream)
+            rc = af.attn_fwd_ex(*args, 0, None, 0, stream.cuda_stream)
             if rc != 0:
-                raise af.AttnError(rc, "attn_fwd")
+                raise af.AttnError(rc, "attn_fwd_ex")
         ms = statistics.median(x[0] for x in time_steps([split], 20, 5, flush, stream))
         ms_whole = statistics.median(x[0] for x in time_steps([whole], 10, 3, flush, stream))
         gbs = w.io_bytes() / (ms * 1e-3) / 1e9
         res[name] = {
-            "shape": f"B={w.B} H={w.H} Sq={w.Sq} Sk={w.Sk} D={w.D} {w.dtype}",
+            "shape": f"B={w.B} H={w.H} Hkv={Hkv} Sq={w.Sq} Sk={w.Sk} D={w.D} {w.dtype}",
             "n_splits": n, "ms": round(ms, 4), "GB/s": round(gbs, 1),
             "frac_of_hbm": round(gbs / hbm, 4),
             "TFLOP/s": round(w.flops(False) / (ms * 1e-3) / 1e12, 1),
@@ -424,6 +428,85 @@ def decode_workloads(names):
         del q, k, v, o, lse, ws
         torch.cuda.empty_cache()
     res["peak_GB/s"] = f"{hbm} ({peak_kind} HBM copy)"
+    return res
+
+
+def softmax_workloads(names):
+    """The standalone row softmax (HBM-bound: x read once, y written once), timed like
+    the rest with a cold L2, as GB/s of those algorithmic bytes."""
+    import attention_forward_18_b200 as af
+    from workloads import SOFTMAX_WORKLOADS, make_rows
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    codes = {"f16": af.ATTN_F16, "bf16": af.ATTN_BF16, "f32": af.SOFTMAX_F32}
+    res = {}
+    for name in names:
+        w = SOFTMAX_WORKLOADS[name]
+        x = make_rows(w.rows, w.n, w.dtype, w.seed, w.scale).to(dev)
+        y = torch.empty_like(x)
+
+        def f():
+            rc = af.row_softmax_raw(x.data_ptr(), y.data_ptr(), w.rows, w.n, codes[w.dtype],
+                                    stream.cuda_stream)
+            if rc != 0:
+                raise af.AttnError(rc, "row_softmax")
+        ms = statistics.median(t[0] for t in time_steps([f], 20, 5, flush, stream))
+        gbs = w.io_bytes() / (ms * 1e-3) / 1e9
+        res[name] = {"shape": f"{w.rows} x {w.n} {w.dtype}", "ms": round(ms, 4),
+                     "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4)}
+        del x, y
+        torch.cuda.empty_cache()
+    res["peak_GB/s"] = f"{hbm} ({peak_kind} HBM copy)"
+    return res
+
+
+def gemm_workloads(names):
+    """The GEMM with the fused bias + activation epilogue (tensor-bound), timed like the
+    rest with a cold L2, as TFLOP/s (2*M*N*K per call) against the measured bf16 peak;
+    torch's cuBLAS linear + activation on the same tensors beside it for context."""
+    import attention_forward_18_b200 as af
+    from workloads import GEMM_WORKLOADS, make_gemm
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    res = {}
+    for name in names:
+        g = GEMM_WORKLOADS[name]
+        a, w, b = (t.to(dev) for t in make_gemm(g.M, g.N, g.K, g.dtype, g.seed))
+        c = torch.empty((g.M, g.N), dtype=a.dtype, device=dev)
+        dcode = af.ATTN_F16 if g.dtype == "f16" else af.ATTN_BF16
+
+        def f():
+            rc = af.gemm_bias_act_raw(a.data_ptr(), w.data_ptr(), b.data_ptr(), c.data_ptr(),
+                                      g.M, g.N, g.K, g.act, dcode, stream.cuda_stream)
+            if rc != 0:
+                raise af.AttnError(rc, "gemm_bias_act")
+
+        def lib():
+            z = torch.nn.functional.linear(a, w, b)
+            if g.act == af.GEMM_ACT_GELU:
+                z = torch.nn.functional.gelu(z)
+            elif g.act == af.GEMM_ACT_RELU:
+                z = torch.relu(z)
+            return z
+        ms = statistics.median(t[0] for t in time_steps([f], 20, 5, flush, stream))
+        ms_lib = statistics.median(t[0] for t in time_steps([lib], 20, 5, flush, stream))
+        tf = g.flops() / (ms * 1e-3) / 1e12
+        res[name] = {"shape": f"M={g.M} N={g.N} K={g.K} {g.dtype} act={g.act}",
+                     "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                     "frac_of_peak": round(tf / peak, 4),
+                     "torch_cublas_TFLOP/s": round(g.flops() / (ms_lib * 1e-3) / 1e12, 1)}
+        status = af.attn_fwd_status(stream)
+        if status != 0:
+            raise af.AttnError(status, f"device status after {name}")
+        del a, w, b, c
+        torch.cuda.empty_cache()
+    res["peak_TFLOP/s"] = f"{peak} ({peak_kind} dense bf16 burst)"
     return res
 
 
@@ -498,6 +581,8 @@ def profile_once(args):
     """One launch per pass of the workload, nothing else on the GPU before it except
     the input copies (a short, self-ending command for ncu)."""
     import attention_forward_18_b200 as af
+    if args.profile_extra:
+        return profile_extra(args.profile_extra)
     w = WORKLOADS[args.workload]
     q, k, v = (t.cuda() for t in make_inputs(w))
     for c in w.causal:
@@ -507,6 +592,43 @@ def profile_once(args):
     if status != 0:
         raise af.AttnError(status, "device status")
     print(json.dumps({"profile_once": w.name, "passes": list(w.causal)}))
+
+
+def profile_extra(spec):
+    """One call of a decode, row-softmax or GEMM workload (its size optionally cut down
+    along its first dimension so an ncu capture stays small)."""
+    import dataclasses
+    import attention_forward_18_b200 as af
+    from workloads import DECODE_WORKLOADS, GEMM_WORKLOADS, SOFTMAX_WORKLOADS, make_gemm, make_rows
+    name, _, cut = spec.partition(":")
+    if name in DECODE_WORKLOADS:
+        w = DECODE_WORKLOADS[name]
+        if cut:
+            w = dataclasses.replace(w, B=int(cut))
+        q, k, v = (t.cuda() for t in make_inputs(w))
+        n = af.ex_default_splits(w.B, w.H, w.kv_heads, w.Sq, w.Sk, af.ATTN_MASK_NONE)
+        af.attention_ex(q, k, v, mask=af.ATTN_MASK_NONE, scale=w.scale, n_splits=n)
+        shape = f"B={w.B} H={w.H} Hkv={w.kv_heads} Sq={w.Sq} Sk={w.Sk} D={w.D} splits={n}"
+    elif name in SOFTMAX_WORKLOADS:
+        w = SOFTMAX_WORKLOADS[name]
+        if cut:
+            w = dataclasses.replace(w, rows=int(cut))
+        af.row_softmax(make_rows(w.rows, w.n, w.dtype, w.seed, w.scale).cuda())
+        shape = f"{w.rows} x {w.n} {w.dtype}"
+    elif name in GEMM_WORKLOADS:
+        g = GEMM_WORKLOADS[name]
+        if cut:
+            g = dataclasses.replace(g, M=int(cut))
+        a, wt, b = (t.cuda() for t in make_gemm(g.M, g.N, g.K, g.dtype, g.seed))
+        af.gemm_bias_act(a, wt, b, g.act)
+        shape = f"M={g.M} N={g.N} K={g.K} {g.dtype} act={g.act}"
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    torch.cuda.synchronize()
+    status = af.attn_fwd_status()
+    if status != 0:
+        raise af.AttnError(status, "device status")
+    print(json.dumps({"profile_once": name, "shape": shape}))
 
 
 def main():
@@ -523,7 +645,10 @@ def main():
         line = cuda_arm(args, world, rank, local)
         if rank == 0 and not args.no_extra:
             line["extra"] = extra_workloads(["C3", "C4", "C5"], world)
-            line["extra"]["decode_splitkv"] = decode_workloads(["DEC1", "DEC2", "DEC3", "DEC4"])
+            line["extra"]["decode_splitkv"] = decode_workloads(
+                ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])
+            line["extra"]["row_softmax"] = softmax_workloads(["SMX1", "SMX2", "SMX3"])
+            line["extra"]["gemm_bias_act"] = gemm_workloads(["GEMM1", "GEMM2", "GEMM3"])
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             w = WORKLOADS[args.workload]
             tf, cores, desc = oracle_sample(w, args.cpu_seconds)

@@ -44,6 +44,16 @@ typedef struct CUstream_st *attn_stream_t;
 /* Element type of Q, K, V and O. */
 typedef enum { ATTN_F16 = 0, ATTN_BF16 = 1 } attn_dtype_t;
 
+/* Mask of attn_fwd_ex.  ATTN_MASK_CAUSAL is the `causal` of attn_fwd: key j visible to
+ * query i iff j <= i (top-left).  ATTN_MASK_CAUSAL_BOTTOM_RIGHT: iff j <= i + Sk - Sq
+ * (the last query sees every key); with Sq > Sk the first Sq - Sk query rows see no key
+ * and get O = 0, LSE = -inf. */
+typedef enum {
+    ATTN_MASK_NONE = 0,
+    ATTN_MASK_CAUSAL = 1,
+    ATTN_MASK_CAUSAL_BOTTOM_RIGHT = 2
+} attn_mask_t;
+
 enum {
     ATTN_OK = 0,
     ATTN_ERR_NULLPTR = -1,   /* q, k, v or o is null                                */
@@ -57,7 +67,8 @@ enum {
     ATTN_ERR_SCALE = -9,     /* scale is NaN or infinite                            */
     ATTN_ERR_ALIAS = -10,    /* o or lse overlaps q, k or v                         */
     ATTN_ERR_DEVICE = -11,   /* no CUDA device, or the current one is not sm_100    */
-    ATTN_ERR_WORKSPACE = -12 /* split pass: workspace smaller than required         */
+    ATTN_ERR_WORKSPACE = -12,/* split pass: workspace smaller than required         */
+    ATTN_ERR_MASK = -13      /* attn_fwd_ex: mask is not an ATTN_MASK_* value       */
 };
 
 /*
@@ -115,6 +126,29 @@ int attn_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float
                      int dtype, int n_splits, void *workspace, size_t workspace_bytes,
                      attn_stream_t stream);
 
+/*
+ * attn_fwd_ex -- the general entry point: grouped K/V heads, the mask choice and the
+ * split-KV option in one call (attn_fwd and attn_fwd_splitkv are special cases).
+ *   H_kv   heads of K and V, a divisor of H: k, v are [B,H_kv,Sk,D] and query head h
+ *          reads K/V head h / (H / H_kv) (grouped-query attention; H_kv = H is plain
+ *          multi-head attention).  The H / H_kv query heads of a group are processed
+ *          together as one sequence of (H / H_kv) * Sq rows, which must be <= 2^24.
+ *   mask   ATTN_MASK_NONE, ATTN_MASK_CAUSAL or ATTN_MASK_CAUSAL_BOTTOM_RIGHT
+ *          (ATTN_ERR_MASK otherwise)
+ *   n_splits  0: the whole pass (workspace may be NULL); 1 .. 1024: the split pass
+ *          with `workspace` as for attn_fwd_splitkv (its size from
+ *          attn_fwd_splitkv_workspace_bytes(B, H, Sq, D, n_splits))
+ * The pages name causal and non-causal attention only; grouped heads and the
+ * bottom-right alignment are this library's options.
+ */
+int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                int B, int H, int H_kv, int Sq, int Sk, int D, int mask, float scale,
+                int dtype, int n_splits, void *workspace, size_t workspace_bytes,
+                attn_stream_t stream);
+
+/* attn_fwd_splitkv_default_splits for attn_fwd_ex's arguments (0 for invalid ones). */
+int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int mask);
+
 /* Bytes of workspace attn_fwd_splitkv needs (0 for invalid arguments). */
 size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_splits);
 
@@ -152,8 +186,9 @@ int attn_fwd_splitkv_noalloc(const void *q, const void *k, const void *v, void *
 
 /*
  * attn_fwd_status -- synchronise `stream`, copy the current device's status word
- * into *device_status (0, or the first ATTN_ERR_* a kernel recorded since the last
- * read) and reset it to 0.  Returns ATTN_OK, ATTN_ERR_NULLPTR or ATTN_ERR_LAUNCH.
+ * into *device_status (0, or the first ATTN_ERR_* a kernel of this library -- the
+ * attention kernels, then the GEMM kernels of gemm_bias_act.h -- recorded since the
+ * last read) and reset it to 0.  Returns ATTN_OK, ATTN_ERR_NULLPTR or ATTN_ERR_LAUNCH.
  */
 int attn_fwd_status(attn_stream_t stream, int *device_status);
 

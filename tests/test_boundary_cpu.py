@@ -1,7 +1,8 @@
-"""The C-ABI library on the CPU: it loads, exports every symbol include/attn_fwd.h
-declares, and rejects bad arguments with the documented codes before any CUDA
-call (no kernel runs here)."""
+"""The C-ABI library on the CPU: it loads, exports every symbol the headers in
+include/ declare, and rejects bad arguments with the documented codes before any
+CUDA call (no kernel runs here)."""
 import ctypes
+import glob
 import os
 import re
 
@@ -10,16 +11,18 @@ import pytest
 import attention_forward_18_b200 as af
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "attn_fwd.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 # fake, never-dereferenced device addresses (16-byte aligned, far apart)
 Q, K, V, O, L = 0x10000000, 0x20000000, 0x30000000, 0x40000000, 0x50000000
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(attn_\w+)\s*\(", text, re.M)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_binding_exports():
@@ -34,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_strerror():
     assert af.abi_version() == 1
-    for code in range(0, -13, -1):
+    for code in range(0, -14, -1):
         msg = af.strerror(code)
         assert msg and msg != "unknown error code", code
     assert af.strerror(12345) == "unknown error code"
@@ -152,3 +155,86 @@ def test_splitkv_default_splits_in_range():
 ])
 def test_splitkv_argument_errors(kw, code):
     assert split_call(**kw) == code
+
+
+def ex_call(**kw):
+    a = dict(q=Q, k=K, v=V, o=O, lse=L, B=2, H=8, H_kv=2, Sq=64, Sk=4096, D=128,
+             mask=af.ATTN_MASK_NONE, scale=0.1, dtype=af.ATTN_BF16, n_splits=0, ws=None,
+             ws_bytes=0)
+    a.update(kw)
+    return af.attn_fwd_ex(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["H_kv"],
+                          a["Sq"], a["Sk"], a["D"], a["mask"], a["scale"], a["dtype"],
+                          a["n_splits"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mask=3), af.ATTN_ERR_MASK),
+    (dict(mask=-1), af.ATTN_ERR_MASK),
+    (dict(H_kv=3), af.ATTN_ERR_SHAPE),          # does not divide H
+    (dict(H_kv=0), af.ATTN_ERR_SHAPE),
+    (dict(H=64, H_kv=1, Sq=1 << 19), af.ATTN_ERR_SHAPE),   # 2^25 packed rows
+    (dict(n_splits=-1), af.ATTN_ERR_SHAPE),
+    (dict(n_splits=2), af.ATTN_ERR_NULLPTR),    # split pass without a workspace
+    (dict(D=96), af.ATTN_ERR_HEADDIM),
+    (dict(o=K + 4096), af.ATTN_ERR_ALIAS),      # inside K (sized with H_kv heads)
+])
+def test_ex_argument_errors(kw, code):
+    assert ex_call(**kw) == code
+
+
+def test_ex_valid_arguments_reach_the_device_check():
+    # no device here: valid arguments fail only at the device check
+    assert ex_call() == af.ATTN_ERR_DEVICE
+    assert ex_call(mask=af.ATTN_MASK_CAUSAL_BOTTOM_RIGHT, H_kv=8) == af.ATTN_ERR_DEVICE
+
+
+def test_ex_default_splits():
+    assert af.ex_default_splits(2, 8, 8, 1, 131072) == af.splitkv_default_splits(2, 8, 1, 131072)
+    # 4 query heads per K/V head are packed into one unit: fewer units, more splits
+    assert af.ex_default_splits(1, 32, 8, 1, 32768) >= af.splitkv_default_splits(1, 32, 1, 32768)
+    # bottom-right causal with one query row sees every key: split like non-causal
+    assert (af.ex_default_splits(1, 8, 8, 1, 131072, af.ATTN_MASK_CAUSAL_BOTTOM_RIGHT) ==
+            af.ex_default_splits(1, 8, 8, 1, 131072, af.ATTN_MASK_NONE))
+    assert af.ex_default_splits(1, 8, 3, 1, 100) == 0
+    assert af.ex_default_splits(1, 8, 8, 1, 100, 5) == 0
+
+
+@pytest.mark.parametrize("args,code", [
+    ((Q, O, 4, 0, af.ATTN_F16), af.ATTN_ERR_SHAPE),
+    ((Q, O, -1, 8, af.ATTN_F16), af.ATTN_ERR_SHAPE),
+    ((Q, O, 4, (1 << 28) + 1, af.ATTN_F16), af.ATTN_ERR_SHAPE),
+    ((Q, O, 4, 8, 3), af.ATTN_ERR_DTYPE),
+    ((None, O, 4, 8, af.ATTN_F16), af.ATTN_ERR_NULLPTR),
+    ((Q + 1, O, 4, 8, af.ATTN_F16), af.ATTN_ERR_ALIGN),
+    ((Q, O + 2, 4, 8, af.SOFTMAX_F32), af.ATTN_ERR_ALIGN),
+    ((Q, Q + 2, 4, 8, af.ATTN_F16), af.ATTN_ERR_ALIAS),     # partial overlap
+    ((Q, O, 0, 8, af.ATTN_F16), af.ATTN_OK),                # no rows: nothing to do
+    ((None, None, 0, 8, af.ATTN_F16), af.ATTN_OK),
+    ((Q, Q, 4, 8, af.ATTN_F16), af.ATTN_ERR_DEVICE),        # in place is allowed
+])
+def test_row_softmax_argument_errors(args, code):
+    x, y, rows, n, dt = args
+    assert af.row_softmax_raw(x, y, rows, n, dt, None) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(a=None), af.ATTN_ERR_NULLPTR),
+    (dict(c=None), af.ATTN_ERR_NULLPTR),
+    (dict(dtype=2), af.ATTN_ERR_DTYPE),
+    (dict(act=3), af.ATTN_ERR_SHAPE),
+    (dict(M=0), af.ATTN_ERR_SHAPE),
+    (dict(N=12), af.ATTN_ERR_SHAPE),            # N not a multiple of 8
+    (dict(K=100), af.ATTN_ERR_SHAPE),           # K not a multiple of 8
+    (dict(a=Q + 8), af.ATTN_ERR_ALIGN),
+    (dict(bias=V + 1), af.ATTN_ERR_ALIGN),
+    (dict(c=Q + 64), af.ATTN_ERR_ALIAS),
+    (dict(c=V - 16), af.ATTN_ERR_ALIAS),        # overlaps the bias
+    (dict(), af.ATTN_ERR_DEVICE),               # valid: fails only at the device check
+    (dict(bias=None), af.ATTN_ERR_DEVICE),
+])
+def test_gemm_argument_errors(kw, code):
+    a = dict(a=Q, w=K, bias=V, c=O, M=300, N=512, K=1024, act=af.GEMM_ACT_GELU,
+             dtype=af.ATTN_BF16)
+    a.update(kw)
+    assert af.gemm_bias_act_raw(a["a"], a["w"], a["bias"], a["c"], a["M"], a["N"], a["K"],
+                                a["act"], a["dtype"], None) == code

@@ -117,21 +117,26 @@ def test_workspace_too_small_is_rejected_on_device():
     assert rc == af.ATTN_ERR_WORKSPACE
 
 
-@pytest.mark.parametrize("name", ["DEC1", "DEC2", "DEC3", "DEC4"])
+@pytest.mark.parametrize("name", ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])
 def test_decode_workloads_in_bench_configuration(name):
-    """The benchmark's decode workloads with the split count the benchmark uses: every
-    row against the oracle (sampled rows for DEC3's 2048 rows x 64K keys)."""
+    """The benchmark's decode workloads with the split count the benchmark uses (DEC5
+    with grouped K/V heads through attn_fwd_ex): every row against the oracle (sampled
+    rows for DEC3's 2048 rows x 64K keys)."""
     from workloads import DECODE_WORKLOADS, make_inputs, sample_rows
     w = DECODE_WORKLOADS[name]
     q, k, v = make_inputs(w)
-    n = af.splitkv_default_splits(w.B, w.H, w.Sq, w.Sk, False)
-    o, lse = run_split(q, k, v, False, w.scale, n)
+    n = af.ex_default_splits(w.B, w.H, w.kv_heads, w.Sq, w.Sk, af.ATTN_MASK_NONE)
+    dq, dk, dv = (t.cuda() for t in (q, k, v))
+    o, lse = af.attention_ex(dq, dk, dv, mask=af.ATTN_MASK_NONE, scale=w.scale, n_splits=n)
+    torch.cuda.synchronize()
+    assert af.attn_fwd_status() == 0
+    o, lse = o.double().cpu().numpy(), lse.double().cpu().numpy()
     qd, kd, vd = q.double().numpy(), k.double().numpy(), v.double().numpy()
     if w.Sq <= 8:
-        o_ref, lse_ref = oracle.attn_ref(qd, kd, vd, False, w.scale)
+        o_ref, lse_ref = oracle.attn_ref_ex(qd, kd, vd, oracle.NO_MASK, w.scale)
         compare(o, lse, o_ref, lse_ref, name)
     else:
         rows = sample_rows(w.B, w.H, w.Sq, 64, seed=w.seed)
-        ro, rl = oracle.attn_ref_rows(qd, kd, vd, rows, False, w.scale)
+        ro, rl = oracle.attn_ref_rows_ex(qd, kd, vd, rows, oracle.NO_MASK, w.scale)
         idx = tuple(np.array(rows).T)
         compare(o[idx], lse[idx], ro, rl, name)

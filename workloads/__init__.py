@@ -30,6 +30,11 @@ class Workload:
     seed: int
     k_scale: float = 1.0
     note: str = ""
+    Hkv: int = 0        # K/V heads (grouped-query attention); 0 means H
+
+    @property
+    def kv_heads(self):
+        return self.Hkv or self.H
 
     @property
     def scale(self):
@@ -43,6 +48,10 @@ class Workload:
         return flops(self.B, self.H, self.Sq, self.Sk, self.D, causal)
 
     def io_bytes(self):
+        if self.kv_heads != self.H:
+            # Q read and O written per query head, K and V read per K/V head
+            return (2 * self.B * self.D * (2 * self.H * self.Sq + 2 * self.kv_heads * self.Sk)
+                    + 4 * self.B * self.H * self.Sq)
         return io_bytes(self.B, self.H, self.Sq, self.Sk, self.D, 2)
 
 
@@ -74,7 +83,91 @@ DECODE_WORKLOADS = {
                      note="64 query rows per head (a block of drafted tokens), 64K keys"),
     "DEC4": Workload("DEC4", 16, 32, 1, 4096, 64, "f16", (False,), 8,
                      note="batch of 16, D=64, 4K keys"),
+    "DEC5": Workload("DEC5", 8, 32, 1, 8192, 128, "bf16", (False,), 9, Hkv=8,
+                     note="grouped heads: 32 query heads on 8 K/V heads, batch 8, 8K keys"),
 }
+
+
+@dataclass(frozen=True)
+class RowWorkload:
+    """A rows x n matrix for the standalone row softmax: i.i.d. N(0, 1) times `scale`
+    (float32 from the seeded generator), rounded RN to `dtype`."""
+    name: str
+    rows: int
+    n: int
+    dtype: str          # "f16", "bf16" or "f32"
+    seed: int
+    scale: float = 1.0
+    note: str = ""
+
+    def io_bytes(self):
+        """Algorithmic HBM bytes of one pass: x read once, y written once."""
+        return 2 * self.rows * self.n * (4 if self.dtype == "f32" else 2)
+
+
+# Row-softmax workloads (the pages give the step no sizes): attention-score rows,
+# vocabulary-sized logits, and rows too long for one CTA's registers.
+SOFTMAX_WORKLOADS = {
+    "SMX1": RowWorkload("SMX1", 32768, 4096, "f16", 11, 4.0,
+                        note="attention-score rows: 32768 rows of 4096, fp16"),
+    "SMX2": RowWorkload("SMX2", 4096, 32000, "bf16", 12, 4.0,
+                        note="vocabulary logits: 4096 rows of 32000, bf16"),
+    "SMX3": RowWorkload("SMX3", 64, 1 << 20, "f32", 13, 8.0,
+                        note="long rows: 64 rows of 2^20, fp32 (two-pass path)"),
+}
+
+TORCH_DTYPES_ALL = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def make_rows(rows, n, dtype, seed, scale=1.0):
+    """Seeded rows x n matrix on the CPU in `dtype` ("f16", "bf16" or "f32")."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    x = torch.randn((rows, n), generator=g, dtype=torch.float32)
+    if scale != 1.0:
+        x = x * scale
+    return x.to(TORCH_DTYPES_ALL[dtype])
+
+
+
+@dataclass(frozen=True)
+class GemmWorkload:
+    """C = act(A W^T + bias): A [M, K], W [N, K], bias [N], i.i.d. N(0, 1) float32 from
+    the seeded generator in the order A, W, bias, A and W scaled by 1/sqrt(sqrt(K)) so
+    the products stay O(1), rounded RN to `dtype`."""
+    name: str
+    M: int
+    N: int
+    K: int
+    dtype: str          # "f16" or "bf16"
+    act: int            # 0 none, 1 GELU, 2 ReLU
+    seed: int
+    note: str = ""
+
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+
+# GEMM workloads (the pages give the tutorial's GEMM no sizes): a square GEMM, an MLP
+# up-projection of 4096 tokens, a short-K layer.
+GEMM_WORKLOADS = {
+    "GEMM1": GemmWorkload("GEMM1", 8192, 8192, 8192, "bf16", 1, 21,
+                          note="square 8192^3, bias + GELU"),
+    "GEMM2": GemmWorkload("GEMM2", 4096, 14336, 4096, "bf16", 1, 22,
+                          note="MLP up-projection: 4096 tokens, 4096 -> 14336, bias + GELU"),
+    "GEMM3": GemmWorkload("GEMM3", 8192, 8192, 1024, "f16", 2, 23,
+                          note="short K: 8192 x 8192 x 1024, bias + ReLU, fp16"),
+}
+
+
+def make_gemm(M, N, K, dtype, seed):
+    """Seeded A [M, K], W [N, K], bias [N] on the CPU in `dtype`."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    s = float(K) ** -0.25
+    a = torch.randn((M, K), generator=g, dtype=torch.float32) * s
+    w = torch.randn((N, K), generator=g, dtype=torch.float32) * s
+    b = torch.randn((N,), generator=g, dtype=torch.float32)
+    t = TORCH_DTYPES[dtype]
+    return a.to(t), w.to(t), b.to(t)
 
 
 def flops(B, H, Sq, Sk, D, causal):
@@ -105,6 +198,11 @@ def make_qkv(B, H, Sq, Sk, D, dtype, seed, k_scale=1.0):
 
 
 def make_inputs(w: Workload):
+    if w.kv_heads != w.H:
+        # Q from the workload's seed, K and V (K/V heads only) from a second stream
+        q, _, _ = make_qkv(w.B, w.H, w.Sq, 1, w.D, w.dtype, w.seed, w.k_scale)
+        _, k, v = make_qkv(w.B, w.kv_heads, 1, w.Sk, w.D, w.dtype, w.seed + 100003, w.k_scale)
+        return q, k, v
     return make_qkv(w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, w.seed, w.k_scale)
 
 
