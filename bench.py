@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of
 # the same kernel build (profiles/attn_fwd_kernel_D64_f16_B4H16S1024_bench_workload.md);
 # a workload without a matching capture reports null.
-NCU_TRAFFIC_BYTES = {"C2-noncausal": 25224960}
+NCU_TRAFFIC_BYTES = {"C2-noncausal": 25225472}
 
 
 def parse():
