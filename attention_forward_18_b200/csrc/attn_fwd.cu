@@ -154,10 +154,10 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
 }
 
-template <int D, int NS, bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
+template <int D, int NS, bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN, bool DEC>
 int launch_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const attn::Params& p, int grid, cudaStream_t stream) {
-    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG, SPLIT, GEN>;
+    auto kern = attn::attn_fwd_kernel<D, NS, BF16, CAUSAL, NEG, SPLIT, GEN, DEC>;
     constexpr int smem = attn::SmemLayout<D, NS>::ALLOC;
     static bool attr_set[kMaxDevices];
     static std::mutex mu;
@@ -186,19 +186,31 @@ constexpr int kStages = (D == 64) ? 5 : 2;
 // the common case carries no per-element sign handling.  The general causal forms
 // (an offset or grouped heads) run their own instantiations too, so plain top-left
 // causal attention keeps the simplest per-row arithmetic.
+//
+// Rows that all fit in query tile 0 (at most 128 packed query rows: decoding) take the
+// DEC instantiations, where both softmax warpgroups work on that tile, on alternate KV
+// tiles.  (Plain top-left causal attention with so few rows sees at most 128 keys, one
+// KV tile: nothing to share, so it has no DEC instantiation.)
+template <int D, bool BF16, bool SPLIT, bool CAUSAL, bool GEN>
+int launch_neg_dec(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const attn::Params& p, int grid, cudaStream_t s) {
+    constexpr int NS = kStages<D>;
+    const bool neg = p.scale_log2 < 0.f;
+    const bool dec = p.Sq <= attn::BM;
+    if (dec && (!CAUSAL || GEN))
+        return neg ? launch_one<D, NS, BF16, CAUSAL, true, SPLIT, GEN, !CAUSAL || GEN>(tq, tk, tv, p, grid, s)
+                   : launch_one<D, NS, BF16, CAUSAL, false, SPLIT, GEN, !CAUSAL || GEN>(tq, tk, tv, p, grid, s);
+    return neg ? launch_one<D, NS, BF16, CAUSAL, true, SPLIT, GEN, false>(tq, tk, tv, p, grid, s)
+               : launch_one<D, NS, BF16, CAUSAL, false, SPLIT, GEN, false>(tq, tk, tv, p, grid, s);
+}
+
 template <int D, bool BF16, bool SPLIT>
 int launch_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const attn::Params& p, int grid, bool causal, cudaStream_t s) {
-    const bool neg = p.scale_log2 < 0.f;
-    constexpr int NS = kStages<D>;
     if (causal && (p.causal_off != 0 || p.sq_head != p.Sq))
-        return neg ? launch_one<D, NS, BF16, true, true, SPLIT, true>(tq, tk, tv, p, grid, s)
-                   : launch_one<D, NS, BF16, true, false, SPLIT, true>(tq, tk, tv, p, grid, s);
-    if (causal)
-        return neg ? launch_one<D, NS, BF16, true, true, SPLIT, false>(tq, tk, tv, p, grid, s)
-                   : launch_one<D, NS, BF16, true, false, SPLIT, false>(tq, tk, tv, p, grid, s);
-    return neg ? launch_one<D, NS, BF16, false, true, SPLIT, false>(tq, tk, tv, p, grid, s)
-               : launch_one<D, NS, BF16, false, false, SPLIT, false>(tq, tk, tv, p, grid, s);
+        return launch_neg_dec<D, BF16, SPLIT, true, true>(tq, tk, tv, p, grid, s);
+    if (causal) return launch_neg_dec<D, BF16, SPLIT, true, false>(tq, tk, tv, p, grid, s);
+    return launch_neg_dec<D, BF16, SPLIT, false, false>(tq, tk, tv, p, grid, s);
 }
 
 template <bool SPLIT>

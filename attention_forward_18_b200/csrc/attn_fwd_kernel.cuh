@@ -337,6 +337,42 @@ __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int S
     return softmax_tile_body<IS_BF16, NEG, false, GEN>(tS, j, 0, c, m_used, l);
 }
 
+// O = 0, LSE = -inf for a row that sees no key (whole pass: 16-bit O; split pass: the
+// fp32 partials of the range).
+template <int D, bool SPLIT>
+__device__ __forceinline__ void write_empty_row(const Params& p, int64_t head_row, int bh,
+                                                int qrow) {
+    if constexpr (SPLIT) {
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        p.ws_lse[head_row * p.Sq + qrow] = -INFINITY;
+    } else {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                              (static_cast<int64_t>(bh) * p.Sq + qrow) * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (p.lse != nullptr) p.lse[static_cast<int64_t>(bh) * p.Sq + qrow] = -INFINITY;
+    }
+}
+
+// 8 normalised output values (columns 8c .. 8c+7) of one row: fp32 partials (split
+// pass) or one rounding to 16 bits.
+template <int D, bool IS_BF16, bool SPLIT>
+__device__ __forceinline__ void store_o8(const Params& p, int64_t head_row, int bh, int qrow,
+                                         int c, const float (&f)[8]) {
+    if constexpr (SPLIT) {
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D + 8 * c);
+        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    } else {
+        uint16_t* o = reinterpret_cast<uint16_t*>(p.o) + (static_cast<int64_t>(bh) * p.Sq + qrow) * D;
+        *reinterpret_cast<uint4*>(o + 8 * c) =
+            make_uint4(pack2<IS_BF16>(f[0], f[1]), pack2<IS_BF16>(f[2], f[3]),
+                       pack2<IS_BF16>(f[4], f[5]), pack2<IS_BF16>(f[6], f[7]));
+    }
+}
+
 // The r-th unit of this CTA in a boustrophedon order over the grid (round r takes
 // units r*G .. r*G+G-1, in reverse CTA order on odd rounds), so with heaviest-first
 // units every CTA's total stays close to the others'.  -1 when none is left.
@@ -350,7 +386,12 @@ __device__ __forceinline__ int unit_of(int r, int n_units) {
 // GEN (causal only): the general causal forms -- a nonzero offset (bottom-right
 // alignment) or grouped query heads packed into one sequence; without it a row's
 // position is its row index and the offset is 0, and no row is ever fully masked.
-template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
+// DEC (decode shapes: every unit's rows fit in query tile 0, so tile 1 would be empty):
+// both softmax warpgroups work on tile 0's rows, warpgroup t on the unit's KV tiles
+// t, t + 2, t + 4, ... with its own running max, sum and O_t accumulator; the epilogue
+// merges the two halves exactly (like a split in two).  Two softmax chains then share
+// each KV tile stream, and only Q tile 0 is loaded.
+template <int D, int NS, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN, bool DEC>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -443,9 +484,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int u = unit_of(r, n_units);
             if (u < 0) break;
             const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
-            const int q0t = w.qp * ROWS_PER_CTA + BM * t;
+            const int q0t = w.qp * ROWS_PER_CTA + (DEC ? 0 : BM * t);
             const int qrow = q0t + row;
-            const int n_t = w.n[t];
+            // DEC: warpgroup t takes the unit's KV tiles t, t + 2, ...
+            const int n_t = DEC ? (w.n[0] + 1 - t) >> 1 : w.n[t];
             int row_vis = qrow, tile_vis_min = q0t;
             if (GEN && n_t > 0) {
                 row_vis = (p.sq_head == p.Sq ? qrow : qrow % p.sq_head) + p.causal_off;
@@ -455,8 +497,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < n_t; ++j, ++it) {
                 if (!(ok = warp_wait(ctx, B_SF(t), it & 1))) break;
                 ptx::tc_fence_after();
+                const int kt = DEC ? 2 * j + t : j;  // the KV tile within the unit's range
                 const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG, GEN>(
-                    tS, j, (w.kv0 + j) * BN, p.Sk, row_vis, tile_vis_min, c_abs, m_used, l);
+                    tS, j, (w.kv0 + kt) * BN, p.Sk, row_vis, tile_vis_min, c_abs, m_used, l);
                 // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
                 // bring it to the new max before PV_t,j adds to it
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -499,6 +542,66 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (u < 0) break;
             const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
             const int64_t head_row = static_cast<int64_t>(w.split) * p.BH + w.bh;
+            if constexpr (DEC) {
+                // tile 0's rows from two halves: O_t, m_t, l_t over KV tiles t, t + 2, ...
+                const int qrow = w.qp * ROWS_PER_CTA + row;
+                const bool store = qrow < p.Sq;
+                const int nt1 = w.n[0] >> 1;
+                if (w.n[0] == 0) {
+                    if (store) write_empty_row<D, SPLIT>(p, head_row, w.bh, qrow);
+                    continue;
+                }
+                if (!(ok = warp_wait(ctx, B_ST(0), ut[0] & 1))) break;
+                if (!(ok = warp_wait(ctx, B_OF(0), ut[0] & 1))) break;
+                if (nt1 > 0) {
+                    if (!(ok = warp_wait(ctx, B_ST(1), ut[1] & 1))) break;
+                    if (!(ok = warp_wait(ctx, B_OF(1), ut[1] & 1))) break;
+                }
+                ptx::tc_fence_after();
+                const float m0 = s_fm[row], l0 = s_fl[row];
+                const float m1 = nt1 > 0 ? s_fm[BM + row] : -INFINITY;
+                const float l1 = nt1 > 0 ? s_fl[BM + row] : 0.f;
+                const float mx = fmaxf(m0, m1);
+                // weights of the halves (0 for a half that saw no key)
+                const float a0 = m0 == -INFINITY ? 0.f : ptx::ex2(m0 - mx);
+                const float a1 = m1 == -INFINITY ? 0.f : ptx::ex2(m1 - mx);
+                const float lt = l0 * a0 + l1 * a1;
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                const float w0 = a0 * inv, w1 = a1 * inv;
+                const float lse_row =
+                    lt > 0.f ? (mx + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+                const uint32_t tO0 = tmem + lane_base + TMEM_O;
+#pragma unroll 1
+                for (int c = 0; c < D / 8; ++c) {
+                    uint32_t o0[8], o1[8];
+                    ptx::tmem_ld8(tO0 + 8 * c, o0);
+                    if (nt1 > 0) ptx::tmem_ld8(tO0 + D + 8 * c, o1);
+                    ptx::tmem_wait_ld();
+                    ptx::reg_fence8(o0);
+                    if (nt1 > 0) ptx::reg_fence8(o1);
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        f[e] = __uint_as_float(o0[e]) * w0 +
+                               (nt1 > 0 ? __uint_as_float(o1[e]) * w1 : 0.f);
+                    if (store) store_o8<D, IS_BF16, SPLIT>(p, head_row, w.bh, qrow, c, f);
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(B_OE(0));
+                    if (nt1 > 0) ptx::mbar_arrive(B_OE(1));
+                }
+                ++ut[0];
+                if (nt1 > 0) ++ut[1];
+                if (store) {
+                    if constexpr (SPLIT)
+                        p.ws_lse[head_row * p.Sq + qrow] = lse_row;
+                    else if (p.lse != nullptr)
+                        p.lse[static_cast<int64_t>(w.bh) * p.Sq + qrow] = lse_row;
+                }
+                continue;
+            }
             for (int t = 0; ok && t < 2; ++t) {
                 const int qrow = w.qp * ROWS_PER_CTA + BM * t + row;
                 const bool store = qrow < p.Sq;
@@ -600,7 +703,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 constexpr uint32_t TILE16 = L::TILE_BYTES >> 4;
                 // S_t = Q_t K^T for the K tile in ring slot `slot`
                 auto issue_s = [&](int t, int slot) {
-                    const uint32_t qd = dq0 + static_cast<uint32_t>(t) * TILE16;
+                    // (DEC: both S accumulators take query tile 0)
+                    const uint32_t qd = dq0 + static_cast<uint32_t>(DEC ? 0 : t) * TILE16;
                     const uint32_t kd = dk0 + static_cast<uint32_t>(slot) * TILE16;
                     const uint32_t d_tmem = tmem + TMEM_S + 128u * t;
                     // K-steps of 16: +32 bytes inside a 128-byte row, +16 KB per 64 columns
@@ -637,7 +741,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint32_t pit[2] = {0, 0};  // P phases per query tile
                 uint32_t ut[2] = {0, 0};   // units with rows per query tile
                 uint32_t nu = 0;           // units so far (Q phases)
-                for (int r = 0; ok; ++r) {
+                // DEC order, KV tile j to accumulator t = j % 2:
+                //   S0,0 S1,1 | PV0,0 S0,2 | PV1,1 S1,3 | PV0,2 S0,4 | ...
+                // each K / V ring position is used by one product.
+                for (int r = 0; DEC && ok; ++r) {
+                    const int u = unit_of(r, n_units);
+                    if (u < 0) break;
+                    const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
+                    const int n = w.n[0];
+                    if (n == 0) continue;  // a range no row of the unit sees
+                    const int nt[2] = {(n + 1) >> 1, n >> 1};
+                    auto slot = [&](int j) { return static_cast<int>((kv + j) % NS); };
+                    auto phase = [&](int j) { return ((kv + j) / NS) & 1u; };
+                    if (!(ok = wait_bounded(ctx, B_QF(0), nu & 1))) break;
+                    for (int j = 0; ok && j < 2 && j < n; ++j) {
+                        if (!(ok = wait_bounded(ctx, B_KF(slot(j)), phase(j)))) break;
+                        ptx::tc_fence_after();
+                        issue_s(j, slot(j));
+                        ptx::mma_commit(B_KE(slot(j)));
+                        if (j == n - 1) ptx::mma_commit(B_QE);  // the unit's last S is issued
+                    }
+                    for (int j = 0; ok && j < n; ++j) {
+                        const int t = j & 1, i = j >> 1;
+                        if (!(ok = wait_bounded(ctx, B_VF(slot(j)), phase(j)))) break;
+                        if (!(ok = wait_bounded(ctx, B_PF(t), pit[t] & 1))) break;
+                        ++pit[t];
+                        // the first P V into O_t overwrites it: the epilogue must have read
+                        // the previous unit's O_t
+                        if (i == 0 && !(ok = wait_bounded(ctx, B_OE(t), (ut[t] & 1) ^ 1))) break;
+                        ptx::tc_fence_after();
+                        issue_pv(t, slot(j), i == 0);
+                        ptx::mma_commit(B_VE(slot(j)));
+                        if (i == nt[t] - 1) ptx::mma_commit(B_OF(t));
+                        if (j + 2 < n) {
+                            if (!(ok = wait_bounded(ctx, B_KF(slot(j + 2)), phase(j + 2)))) break;
+                            ptx::tc_fence_after();
+                            issue_s(t, slot(j + 2));
+                            ptx::mma_commit(B_KE(slot(j + 2)));
+                            if (j + 2 == n - 1) ptx::mma_commit(B_QE);  // last S issued
+                        }
+                    }
+                    for (int t = 0; t < 2; ++t) ut[t] += nt[t] > 0 ? 1u : 0u;
+                    kv += static_cast<uint32_t>(n);
+                    ++nu;
+                }
+                for (int r = 0; !DEC && ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
                     const Unit w = decode_unit<CAUSAL, SPLIT, GEN>(u, p);
@@ -706,9 +854,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int n_max = max(w.n[0], w.n[1]);
                     if (n_max == 0) continue;  // nothing to load (the MMA skips it too)
                     // Q_0, Q_1 are free once the previous unit's S MMAs completed
+                    // (DEC: only Q_0 is used)
                     if (!(ok = wait_bounded(ctx, B_QE, (nu & 1) ^ 1))) break;
                     if (load_q) {
-                        for (int t = 0; t < 2; ++t) {
+                        for (int t = 0; t < (DEC ? 1 : 2); ++t) {
                             ptx::mbar_arrive_expect_tx(B_QF(t), L::TILE_BYTES);
                             for (int c = 0; c < L::NCH; ++c)
                                 ptx::tma_load_3d(sQ + t * L::TILE_BYTES + c * CHUNK_BYTES, &tm_q,
@@ -739,7 +888,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // Let every copy this thread started land before the CTA can exit.
                 if (last_q >= 0) {
                     wait_drain(B_QF(0), static_cast<uint32_t>(last_q) & 1);
-                    wait_drain(B_QF(1), static_cast<uint32_t>(last_q) & 1);
+                    if (!DEC) wait_drain(B_QF(1), static_cast<uint32_t>(last_q) & 1);
                 }
                 for (int64_t q = (last_k - NS + 1 > 0 ? last_k - NS + 1 : 0); q <= last_k; ++q)
                     wait_drain(B_KF(static_cast<int>(q % NS)), (q / NS) & 1);
