@@ -11,9 +11,8 @@
 //   * longer rows (or rows whose length breaks 16-byte alignment): a cluster of up to
 //     8 CTAs per row, each CTA a contiguous slice, in two passes: an online max / sum
 //     of the slice, an exchange of the CTAs' (max, sum) pairs through distributed
-//     shared memory, then the normalised output.  The clusters are persistent and
-//     few (about one CTA per SM), so the rows in flight fit in L2 and the second read
-//     of a slice is served from L2.
+//     shared memory, then the normalised output (four 16-byte loads in flight per
+//     thread in each pass).  The slice is read twice.
 // Grids are persistent: (resident CTAs per SM) x (SMs), each group walking rows.
 // exp is ex2 on d = x - max (the difference first, so |d| carries the only rounding),
 // the sum accumulates in fp32 and the output is rounded once.
@@ -306,12 +305,23 @@ __global__ void __launch_bounds__(1024) softmax_cluster_rows(const void* __restr
     for (int64_t r = blockIdx.x / csize; r < rows; r += n_clusters) {
         float m = -INFINITY, s = 0.f;
         if constexpr (VEC) {
+            // four 16-byte loads in flight per thread before they are used
             const uint4* src = reinterpret_cast<const uint4*>(x) + r * units;
-            for (int u = beg + tid; u < end; u += blockDim.x) {
-                float v[EPV];
-                C::unpack(__ldcg(src + u), v);
+            const int step = static_cast<int>(blockDim.x);
+            for (int u0 = beg + tid; u0 < end; u0 += 4 * step) {
+                uint4 c[4];
 #pragma unroll
-                for (int e = 0; e < EPV; ++e) online_add(m, s, v[e]);
+                for (int i = 0; i < 4; ++i)
+                    c[i] = u0 + i * step < end ? __ldcg(src + u0 + i * step) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (u0 + i * step < end) {
+                        float v[EPV];
+                        C::unpack(c[i], v);
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) online_add(m, s, v[e]);
+                    }
+                }
             }
         } else {
             for (int u = beg + tid; u < end; u += blockDim.x) online_add(m, s, E::get(x, r * n + u));
@@ -351,12 +361,23 @@ __global__ void __launch_bounds__(1024) softmax_cluster_rows(const void* __restr
         if constexpr (VEC) {
             const uint4* src = reinterpret_cast<const uint4*>(x) + r * units;
             uint4* dst = reinterpret_cast<uint4*>(y) + r * units;
-            for (int u = beg + tid; u < end; u += blockDim.x) {
-                float v[EPV];
-                C::unpack(__ldcs(src + u), v);
+            const int step = static_cast<int>(blockDim.x);
+            for (int u0 = beg + tid; u0 < end; u0 += 4 * step) {
+                uint4 c[4];
 #pragma unroll
-                for (int e = 0; e < EPV; ++e) v[e] = attn::ptx::ex2((v[e] - m) * kLog2e) * inv;
-                __stcs(dst + u, C::pack(v));
+                for (int i = 0; i < 4; ++i)
+                    c[i] = u0 + i * step < end ? __ldcs(src + u0 + i * step) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (u0 + i * step < end) {
+                        float v[EPV];
+                        C::unpack(c[i], v);
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e)
+                            v[e] = attn::ptx::ex2((v[e] - m) * kLog2e) * inv;
+                        __stcs(dst + u0 + i * step, C::pack(v));
+                    }
+                }
             }
         } else {
             for (int u = beg + tid; u < end; u += blockDim.x)
@@ -417,34 +438,41 @@ int launch_cta(const void* x, void* y, int64_t rows, int chunks, int sms, cudaSt
     return ATTN_OK;
 }
 
-// Cluster size: one CTA per 64 KB of row, up to 8 (the portable limit); threads: up to
-// 1024, fewer for short rows.  Grid: as many clusters as can be resident at once, at
-// most one per row.
+// Cluster size: one CTA per 64 KB of row, up to 8 (the portable limit; clusters of 16
+// measured slower here); threads: up to 1024, fewer for short rows.  Grid: as many
+// clusters as can be resident at once, at most one per row.  (Capping the rows in
+// flight so that the second pass reads from L2 also measured slower: it idles SMs.)
 template <int DT, bool VEC>
 int launch_cluster(const void* x, void* y, int64_t rows, int n, int sms, cudaStream_t s) {
     const int64_t bytes = static_cast<int64_t>(n) * Elem<DT>::kBytes;
-    int csize = 1;
-    while (csize < 8 && bytes > static_cast<int64_t>(csize) * 65536) csize *= 2;
-    const int64_t per_cta = (static_cast<int64_t>(n) + csize - 1) / csize;
-    const int threads = per_cta >= 1024 ? 1024 : static_cast<int>((per_cta + 31) / 32 * 32);
     auto k = softmax_cluster_rows<DT, VEC>;
+    constexpr int cmax = 8;
+    int csize = 1;
+    while (csize < cmax && bytes > static_cast<int64_t>(csize) * 65536) csize *= 2;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(static_cast<unsigned>(threads));
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     int max_clusters = 0;
-    cfg.gridDim = dim3(static_cast<unsigned>(csize));
-    if (cudaOccupancyMaxActiveClusters(&max_clusters, k, &cfg) != cudaSuccess || max_clusters < 1) {
-        cudaGetLastError();
-        max_clusters = sms / csize > 0 ? sms / csize : 1;
+    for (;; csize /= 2) {
+        const int64_t per_cta = (static_cast<int64_t>(n) + csize - 1) / csize;
+        const int threads = per_cta >= 1024 ? 1024 : static_cast<int>((per_cta + 31) / 32 * 32);
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg = cudaLaunchConfig_t{};
+        cfg.blockDim = dim3(static_cast<unsigned>(threads));
+        cfg.gridDim = dim3(static_cast<unsigned>(csize));
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, k, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            max_clusters = 0;
+        }
+        if (max_clusters >= 1 || csize == 1) break;  // a cluster this size fits, or none
     }
+    if (max_clusters < 1) max_clusters = sms;
     const int64_t clusters = rows < max_clusters ? rows : max_clusters;
     cfg.gridDim = dim3(static_cast<unsigned>(clusters * csize));
     if (cudaLaunchKernelEx(&cfg, k, x, y, rows, n) != cudaSuccess) {
