@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 continue;
             }
-            for (int t = 0; ok && t < 2; ++t) {
+            if constexpr (!DEC) for (int t = 0; ok && t < 2; ++t) {
                 const int qrow = w.qp * ROWS_PER_CTA + BM * t + row;
                 const bool store = qrow < p.Sq;
                 if (w.n[t] == 0) {
