@@ -379,6 +379,59 @@ def extra_workloads(af_names, world):
     return res
 
 
+def graph_launches(names, reps=20):
+    """C1 / C2 per launch inside a captured CUDA graph of `reps` back-to-back launches
+    of each pass (launch overhead amortised; inputs resident and, at these sizes, warm
+    in L2 after the first launch -- stated in the line)."""
+    import attention_forward_18_b200 as af
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, _ = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    res = {}
+    stream = torch.cuda.Stream(dev)
+    for name in names:
+        w = WORKLOADS[name]
+        q, k, v = (t.to(dev) for t in make_inputs(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+        dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
+        for c in w.causal:
+            def f(c=c):
+                rc = af.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), w.B, w.H, w.Sq, w.Sk, w.D, int(c), w.scale,
+                                 dcode, stream.cuda_stream)
+                if rc != 0:
+                    raise af.AttnError(rc, "attn_fwd")
+            with torch.cuda.stream(stream):
+                f()  # first call outside the capture (one-time set-up)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    f()
+            times = []
+            with torch.cuda.stream(stream):
+                for _ in range(5):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    g.replay()  # on the current stream: `stream`
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    times.append(e0.elapsed_time(e1) / reps)
+            ms = statistics.median(times)
+            tf = w.flops(c) / (ms * 1e-3) / 1e12
+            res[f"{name}{'-causal' if c else ''}"] = {
+                "ms_per_launch": round(ms, 5), "TFLOP/s": round(tf, 1),
+                "frac_of_peak": round(tf / peak, 4),
+                "note": f"{reps} launches per graph replay, L2 warm"}
+            del g
+        status = af.attn_fwd_status()
+        if status != 0:
+            raise af.AttnError(status, f"device status after {name}")
+    return res
+
+
 def decode_workloads(names):
     """The split-KV pass on decode-shaped workloads (HBM-bound: K and V are read once,
     the score work is small), timed like the rest with a cold L2; the whole pass on the
@@ -645,6 +698,7 @@ def main():
         line = cuda_arm(args, world, rank, local)
         if rank == 0 and not args.no_extra:
             line["extra"] = extra_workloads(["C3", "C4", "C5"], world)
+            line["extra"]["cuda_graph"] = graph_launches(["C1", "C2"])
             line["extra"]["decode_splitkv"] = decode_workloads(
                 ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])
             line["extra"]["row_softmax"] = softmax_workloads(["SMX1", "SMX2", "SMX3"])
