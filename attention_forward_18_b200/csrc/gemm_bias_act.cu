@@ -33,26 +33,37 @@ namespace gemm {
 
 namespace ptx = attn::ptx;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;           // 16 KB
+constexpr int BN = 256, BK = 64;
 constexpr int B_BYTES = BN * BK * 2;           // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KB
-constexpr int NUM_THREADS = 384;
-constexpr int EPI_WARP0 = 4, EPI_WARPS = 8;
+constexpr int EPI_WARP0 = 4;
 constexpr int GROUP_M = 8;
-constexpr uint32_t TMEM_COLS = 512;            // two 256-column accumulators
+constexpr uint32_t TMEM_COLS = 512;
+
+// Tile shapes.  MH = 1: 128 x 256 tiles, a 4-stage ring of 48 KB, two 256-column
+// accumulators (the epilogue of one tile overlaps the next tile's products).  MH = 2:
+// 256 x 256 tiles as two M = 128 halves sharing each W tile, a 3-stage ring of 64 KB,
+// one accumulator of two halves (all 512 columns), so a third less A/W traffic per
+// FLOP at the price of an epilogue the next tile waits for (used for long K).
+template <int MH>
+struct Cfg {
+    static constexpr int BM = 128 * MH;
+    static constexpr int STAGES = MH == 1 ? 4 : 3;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int EPI_WARPS = 8 * MH;
+    static constexpr int NUM_THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+    static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+    // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+    static constexpr int NBAR = 2 * STAGES + 5;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align to 1024
+    static_assert(2 * SMEM_BYTES > 232448, "one CTA per SM (it takes all of TMEM)");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_LIMIT_NS = 500000000ull;
 constexpr int STATUS_TIMEOUT = -8;             // ATTN_ERR_TIMEOUT
 
-// shared memory: ring | barriers | tmem slot, error flag
-constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-// full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
-constexpr int NBAR = 2 * STAGES + 5;
-constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
-static_assert(2 * SMEM_BYTES > 232448, "one CTA per SM (it takes all of TMEM)");
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 struct Params {
     void* c;              // [M, N] 16-bit
@@ -131,10 +142,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     else return ptx::pack_f16x2(lo, hi);
 }
 
-template <bool IS_BF16, int ACT, bool HAS_BIAS>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <bool IS_BF16, int ACT, bool HAS_BIAS, int MH>
+__global__ void __launch_bounds__(Cfg<MH>::NUM_THREADS, 1)
     gemm_bias_act_kernel(const __grid_constant__ CUtensorMap tm_a,
                          const __grid_constant__ CUtensorMap tm_w, const Params p) {
+    using C = Cfg<MH>;
+    constexpr int BM = C::BM, STAGES = C::STAGES, A_BYTES = C::A_BYTES;
+    constexpr int STAGE_BYTES = C::STAGE_BYTES, EPI_WARPS = C::EPI_WARPS;
+    constexpr int BAR_OFF = C::BAR_OFF, MISC_OFF = C::MISC_OFF;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = ptx::smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -206,27 +221,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 1) {
         // ================================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_f16(IS_BF16 ? 1u : 0u, BM, BN, 0);
+            constexpr uint32_t idesc = ptx::idesc_f16(IS_BF16 ? 1u : 0u, 128, BN, 0);
             constexpr uint32_t hi = ptx::smem_desc_hi_sw128(1024);
             uint32_t it = 0, i = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++i) {
-                const int ab = static_cast<int>(i & 1u);
-                if (!(ok = wait_bounded(ctx, B_AE(ab), ((i >> 1) & 1u) ^ 1u))) break;
+                // MH = 1: accumulator i % 2, used every other tile; MH = 2: the one
+                // accumulator (both halves), used every tile
+                const int ab = MH == 1 ? static_cast<int>(i & 1u) : 0;
+                const uint32_t use = MH == 1 ? (i >> 1) : i;
+                if (!(ok = wait_bounded(ctx, B_AE(ab), (use & 1u) ^ 1u))) break;
                 ptx::tc_fence_after();
-                const uint32_t d = tmem + static_cast<uint32_t>(ab) * BN;
                 for (int kb = 0; kb < p.num_k; ++kb, ++it) {
                     const int s = static_cast<int>(it % STAGES);
                     if (!(ok = wait_bounded(ctx, B_FULL(s), (it / STAGES) & 1u))) break;
                     ptx::tc_fence_after();
                     const uint32_t sa = sbase + s * STAGE_BYTES;
-                    const uint32_t a_lo = ptx::smem_desc_lo(sa, 16);
                     const uint32_t b_lo = ptx::smem_desc_lo(sa + A_BYTES, 16);
-                    // K steps of 16 elements: +32 bytes inside the 128-byte swizzled row
-                    ptx::mma_ss_off<0, 0>(d, a_lo, b_lo, hi, idesc, kb > 0 ? 1u : 0u);
-                    ptx::mma_ss_off<2, 2>(d, a_lo, b_lo, hi, idesc, 1u);
-                    ptx::mma_ss_off<4, 4>(d, a_lo, b_lo, hi, idesc, 1u);
-                    ptx::mma_ss_off<6, 6>(d, a_lo, b_lo, hi, idesc, 1u);
+#pragma unroll
+                    for (int h = 0; h < MH; ++h) {
+                        // half h: rows 128h.. of the A tile (16 KB further), columns
+                        // 256(ab + h) of tensor memory
+                        const uint32_t d = tmem + static_cast<uint32_t>(ab + h) * BN;
+                        const uint32_t a_lo = ptx::smem_desc_lo(sa + h * 16384, 16);
+                        // K steps of 16 elements: +32 bytes inside the 128-byte row
+                        ptx::mma_ss_off<0, 0>(d, a_lo, b_lo, hi, idesc, kb > 0 ? 1u : 0u);
+                        ptx::mma_ss_off<2, 2>(d, a_lo, b_lo, hi, idesc, 1u);
+                        ptx::mma_ss_off<4, 4>(d, a_lo, b_lo, hi, idesc, 1u);
+                        ptx::mma_ss_off<6, 6>(d, a_lo, b_lo, hi, idesc, 1u);
+                    }
                     ptx::mma_commit(B_EMPTY(s));
                 }
                 if (!ok) break;
@@ -239,25 +262,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
     } else if (warp >= EPI_WARP0) {
         // ================================================================ epilogue
-        const int q = warp & 3;                   // TMEM lane quarter
-        const int half = (warp - EPI_WARP0) >> 2;  // column half of the tile
+        const int q = warp & 3;                          // TMEM lane quarter
+        const int half = ((warp - EPI_WARP0) >> 2) & 1;  // column half of the tile
+        const int mh = (warp - EPI_WARP0) >> 3;          // MH = 2: the M half
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint32_t i = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++i) {
             int mb, nb;
             tile_coords(t, p, mb, nb);
-            const int ab = static_cast<int>(i & 1u);
-            if (!(ok = warp_wait(ctx, B_AF(ab), (i >> 1) & 1u))) break;
+            const int ab = MH == 1 ? static_cast<int>(i & 1u) : 0;
+            const uint32_t use = MH == 1 ? (i >> 1) : i;
+            if (!(ok = warp_wait(ctx, B_AF(ab), use & 1u))) break;
             ptx::tc_fence_after();
-            const int row = mb * BM + q * 32 + lane;
+            const int row = mb * BM + mh * 128 + q * 32 + lane;
             const bool row_ok = row < p.M;
             uint16_t* crow = reinterpret_cast<uint16_t*>(p.c) + static_cast<int64_t>(row) * p.N;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 const int col0 = nb * BN + half * 128 + c * 32;
                 uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_base + static_cast<uint32_t>(ab * BN + half * 128 + c * 32), v);
+                ptx::tmem_ld32(tmem + lane_base +
+                                   static_cast<uint32_t>((ab + mh) * BN + half * 128 + c * 32), v);
                 ptx::tmem_wait_ld();
                 ptx::reg_fence32(v);
 #pragma unroll
@@ -359,32 +385,33 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
-template <bool BF16, int ACT, bool BIAS>
+template <bool BF16, int ACT, bool BIAS, int MH>
 int launch(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p, int grid,
            cudaStream_t s) {
-    auto k = gemm::gemm_bias_act_kernel<BF16, ACT, BIAS>;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::SMEM_BYTES) !=
+    using C = gemm::Cfg<MH>;
+    auto k = gemm::gemm_bias_act_kernel<BF16, ACT, BIAS, MH>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
         cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }
-    k<<<grid, gemm::NUM_THREADS, gemm::SMEM_BYTES, s>>>(ta, tw, p);
+    k<<<grid, C::NUM_THREADS, C::SMEM_BYTES, s>>>(ta, tw, p);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-template <bool BF16, int ACT>
+template <bool BF16, int ACT, int MH>
 int launch_bias(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p, int grid,
                 cudaStream_t s) {
-    return p.bias ? launch<BF16, ACT, true>(ta, tw, p, grid, s)
-                  : launch<BF16, ACT, false>(ta, tw, p, grid, s);
+    return p.bias ? launch<BF16, ACT, true, MH>(ta, tw, p, grid, s)
+                  : launch<BF16, ACT, false, MH>(ta, tw, p, grid, s);
 }
 
-template <bool BF16>
+template <bool BF16, int MH>
 int launch_act(const CUtensorMap& ta, const CUtensorMap& tw, const gemm::Params& p, int act,
                int grid, cudaStream_t s) {
-    if (act == GEMM_ACT_GELU) return launch_bias<BF16, GEMM_ACT_GELU>(ta, tw, p, grid, s);
-    if (act == GEMM_ACT_RELU) return launch_bias<BF16, GEMM_ACT_RELU>(ta, tw, p, grid, s);
-    return launch_bias<BF16, GEMM_ACT_NONE>(ta, tw, p, grid, s);
+    if (act == GEMM_ACT_GELU) return launch_bias<BF16, GEMM_ACT_GELU, MH>(ta, tw, p, grid, s);
+    if (act == GEMM_ACT_RELU) return launch_bias<BF16, GEMM_ACT_RELU, MH>(ta, tw, p, grid, s);
+    return launch_bias<BF16, GEMM_ACT_NONE, MH>(ta, tw, p, grid, s);
 }
 
 int run(const void* a, const void* w, const void* bias, void* c, int M, int N, int K, int act,
@@ -404,8 +431,15 @@ int run(const void* a, const void* w, const void* bias, void* c, int M, int N, i
     const int sms = device_sms();
     if (sms < 1) return ATTN_ERR_DEVICE;
     const bool bf16 = dtype == ATTN_BF16;
+    // 256-row tiles (a third less operand traffic, but an epilogue the next tile waits
+    // for) pay off once a tile's products dwarf its epilogue: measured on B200, from
+    // K = 8192 with the GELU epilogue (+9 % at 8192^3, -7 % at K = 4096) and from
+    // K = 4096 without it (+3-9 %).  Flags 2 / 4 force the 128- / 256-row tiles.
+    const bool wide = M > 128 && K >= (act == GEMM_ACT_GELU ? 8192 : 4096);
+    const int mh = (flags & 2u) ? 1 : (flags & 4u) ? 2 : wide ? 2 : 1;
+    const int BM = 128 * mh;
     CUtensorMap ta, tw;
-    if (!encode_2d(&ta, a, K, M, gemm::BM, bf16) || !encode_2d(&tw, w, K, N, gemm::BN, bf16))
+    if (!encode_2d(&ta, a, K, M, BM, bf16) || !encode_2d(&tw, w, K, N, gemm::BN, bf16))
         return ATTN_ERR_TENSORMAP;
     gemm::Params p;
     p.c = c;
@@ -413,16 +447,19 @@ int run(const void* a, const void* w, const void* bias, void* c, int M, int N, i
     p.M = M;
     p.N = N;
     p.K = K;
-    p.num_m = (M + gemm::BM - 1) / gemm::BM;
+    p.num_m = (M + BM - 1) / BM;
     p.num_n = (N + gemm::BN - 1) / gemm::BN;
     p.num_k = (K + gemm::BK - 1) / gemm::BK;
     const int64_t tiles = static_cast<int64_t>(p.num_m) * p.num_n;
     if (tiles > INT_MAX) return ATTN_ERR_SHAPE;
     p.num_tiles = static_cast<int>(tiles);
-    p.flags = flags;
+    p.flags = flags & 1u;
     const int grid = p.num_tiles < sms ? p.num_tiles : sms;
-    return bf16 ? launch_act<true>(ta, tw, p, act, grid, stream)
-                : launch_act<false>(ta, tw, p, act, grid, stream);
+    if (mh == 2)
+        return bf16 ? launch_act<true, 2>(ta, tw, p, act, grid, stream)
+                    : launch_act<false, 2>(ta, tw, p, act, grid, stream);
+    return bf16 ? launch_act<true, 1>(ta, tw, p, act, grid, stream)
+                : launch_act<false, 1>(ta, tw, p, act, grid, stream);
 }
 
 }  // namespace
@@ -454,7 +491,7 @@ int gemm_bias_act(const void* a, const void* w, const void* bias, void* c, int M
 int gemm_bias_act_debug(const void* a, const void* w, const void* bias, void* c, int M, int N,
                         int K, int act, int dtype, attn_stream_t stream, unsigned flags) {
     return run(a, w, bias, c, M, N, K, act, dtype, reinterpret_cast<cudaStream_t>(stream),
-               flags & 1u);
+               flags & 7u);
 }
 
 }  // extern "C"

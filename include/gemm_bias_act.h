@@ -52,8 +52,9 @@ int gemm_bias_act(const void *a, const void *w, const void *bias, void *c, int M
 /*
  * gemm_bias_act_debug -- gemm_bias_act with kernel debug flags, for the tests.  Flag 1
  * makes the TMA producer skip its loads so the MMA warp's first wait runs out: the
- * call must end with ATTN_ERR_TIMEOUT in the status word, not hang.  Flag 0 is
- * gemm_bias_act.
+ * call must end with ATTN_ERR_TIMEOUT in the status word, not hang.  Flag 2 forces the
+ * 128-row output tiles, flag 4 the 256-row tiles (gemm_bias_act picks by K).  Flag 0
+ * is gemm_bias_act.
  */
 int gemm_bias_act_debug(const void *a, const void *w, const void *bias, void *c, int M,
                         int N, int K, int act, int dtype, attn_stream_t stream,

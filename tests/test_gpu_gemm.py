@@ -90,6 +90,12 @@ def test_timeout_is_reported_and_the_context_survives():
     assert rc == af.ATTN_OK
     assert af.attn_fwd_status() == af.ATTN_ERR_TIMEOUT
     assert af.attn_fwd_status() == 0
+    # the same with the 256-row tiles (flag 4)
+    rc = af.gemm_bias_act_raw(da.data_ptr(), dw.data_ptr(), db.data_ptr(), c.data_ptr(), 256,
+                              512, 128, af.GEMM_ACT_NONE, af.ATTN_BF16,
+                              torch.cuda.current_stream().cuda_stream, flags=1 | 4)
+    assert rc == af.ATTN_OK
+    assert af.attn_fwd_status() == af.ATTN_ERR_TIMEOUT
     c = af.gemm_bias_act(da, dw, db, af.GEMM_ACT_NONE)
     torch.cuda.synchronize()
     check(c, a, w, b, af.GEMM_ACT_NONE, "bf16", "after timeout")
@@ -109,3 +115,21 @@ def test_benchmark_workloads_sampled_rows(name):
     rows = np.unique(np.concatenate([[0, g.M - 1], np.arange(127, 1024, 128),
                                      np.arange(128, 1024, 128), rng.choice(g.M, 8)]))
     check(c, a, w, b, g.act, g.dtype, name, rows=rows)
+
+
+@pytest.mark.parametrize("tiles", [2, 4])
+@pytest.mark.parametrize("M,N,K", [(257, 264, 2048), (1000, 512, 64), (128, 1024, 4096),
+                                   (384, 256, 136)])
+def test_both_tile_shapes(M, N, K, tiles):
+    """Debug flag 2 / 4 forces the 128-row / 256-row output tiles: both give the oracle's
+    result on tile-aligned and ragged shapes (the default picks by K)."""
+    a, w, b = make_gemm(M, N, K, "bf16", seed=M + N + K + tiles)
+    da, dw, db = a.cuda(), w.cuda(), b.cuda()
+    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    rc = af.gemm_bias_act_raw(da.data_ptr(), dw.data_ptr(), db.data_ptr(), c.data_ptr(), M, N,
+                              K, af.GEMM_ACT_GELU, af.ATTN_BF16,
+                              torch.cuda.current_stream().cuda_stream, flags=tiles)
+    assert rc == af.ATTN_OK
+    torch.cuda.synchronize()
+    assert af.attn_fwd_status() == 0
+    check(c, a, w, b, af.GEMM_ACT_GELU, "bf16", f"{M}x{N}x{K} tiles flag {tiles}")
