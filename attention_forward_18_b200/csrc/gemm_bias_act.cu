@@ -10,8 +10,9 @@
 //                next;
 //   warp 2       tensor-memory allocation / release;
 //   warps 4..11  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lane
-//                quarter w % 4, column half (w - 4) / 4), + bias, activation in fp32,
-//                one rounding to 16 bits, 16-byte stores.
+//                quarter w % 4, column half (w - 4) / 4), + bias, activation in fp32
+//                (GELU through a published rational-exponential form of erf), one
+//                rounding to 16 bits, 16-byte stores.
 // Output tiles are visited in groups of 8 M-blocks (N-blocks inner within a group) so
 // the CTAs running at one time share their A and W tiles in L2.
 // Every wait is bounded (2 s); a timeout records ATTN_ERR_TIMEOUT in this file's
@@ -122,9 +123,31 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int
     nb = r / rows;
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// GELU(z) = 0.5 z (1 + erf(z / sqrt 2)) with erf from Abramowitz and Stegun, formula
+// 7.1.26: for x >= 0, erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) e^(-x^2),
+// t = 1 / (1 + p x), absolute error <= 1.5e-7.  The bracket is erfc(x), so for z < 0
+// the factor 1 + erf = erfc(|x|) comes without cancellation; for z >= 0 it is 2 - erfc.
+// Absolute error of the result <= 0.5 |z| (1.5e-7 + a few fp32 roundings).
+__device__ __forceinline__ float gelu(float z) {
+    const float x = fabsf(z) * 0.70710678118654752f;
+    const float t = rcp_approx(fmaf(0.3275911f, x, 1.f));
+    float poly = fmaf(1.061405429f, t, -1.453152027f);
+    poly = fmaf(poly, t, 1.421413741f);
+    poly = fmaf(poly, t, -0.284496736f);
+    poly = fmaf(poly, t, 0.254829592f) * t;
+    const float erfc_x = poly * ptx::ex2(-x * x * 1.4426950408889634f);
+    return 0.5f * z * (z >= 0.f ? 2.f - erfc_x : erfc_x);
+}
+
 template <int ACT>
 __device__ __forceinline__ float activate(float z) {
-    if constexpr (ACT == GEMM_ACT_GELU) return 0.5f * z * (1.f + erff(z * 0.70710678118654752f));
+    if constexpr (ACT == GEMM_ACT_GELU) return gelu(z);
     else if constexpr (ACT == GEMM_ACT_RELU) return fmaxf(z, 0.f);
     else return z;
 }
