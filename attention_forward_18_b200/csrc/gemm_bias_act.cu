@@ -152,11 +152,16 @@ __device__ __forceinline__ float activate(float z) {
     else return z;
 }
 
+// The low / high 16-bit value of a packed pair, as fp32.
 template <bool IS_BF16>
-__device__ __forceinline__ float load16(const void* p, int i) {
-    const uint16_t b = reinterpret_cast<const uint16_t*>(p)[i];
-    if constexpr (IS_BF16) return __uint_as_float(static_cast<uint32_t>(b) << 16);
-    else return __half2float(__ushort_as_half(b));
+__device__ __forceinline__ float unpack_lo(uint32_t w) {
+    if constexpr (IS_BF16) return __uint_as_float(w << 16);
+    else return __half2float(__ushort_as_half(static_cast<uint16_t>(w & 0xffffu)));
+}
+template <bool IS_BF16>
+__device__ __forceinline__ float unpack_hi(uint32_t w) {
+    if constexpr (IS_BF16) return __uint_as_float(w & 0xffff0000u);
+    else return __half2float(__ushort_as_half(static_cast<uint16_t>(w >> 16)));
 }
 
 template <bool IS_BF16>
@@ -285,6 +290,7 @@ __global__ void __launch_bounds__(Cfg<MH>::NUM_THREADS, 1)
         __syncwarp();
     } else if (warp >= EPI_WARP0) {
         // ================================================================ epilogue
+        const bool bias_vec = (reinterpret_cast<uintptr_t>(p.bias) & 15u) == 0;
         const int q = warp & 3;                          // TMEM lane quarter
         const int half = ((warp - EPI_WARP0) >> 2) & 1;  // column half of the tile
         const int mh = (warp - EPI_WARP0) >> 3;          // MH = 2: the M half
@@ -314,13 +320,29 @@ __global__ void __launch_bounds__(Cfg<MH>::NUM_THREADS, 1)
                     const int cg = col0 + 8 * g;  // N is a multiple of 8: groups are whole
                     if (cg >= p.N) continue;
                     uint32_t w[4];
+                    // the group's 8 bias values: one 16-byte load when the bias is
+                    // 16-byte aligned (cg is a multiple of 8), else one by one
+                    uint32_t bw[4] = {0u, 0u, 0u, 0u};
+                    if constexpr (HAS_BIAS) {
+                        if (bias_vec) {
+                            const uint4 bv = *reinterpret_cast<const uint4*>(
+                                reinterpret_cast<const uint16_t*>(p.bias) + cg);
+                            bw[0] = bv.x, bw[1] = bv.y, bw[2] = bv.z, bw[3] = bv.w;
+                        } else {
+                            const uint16_t* bp = reinterpret_cast<const uint16_t*>(p.bias) + cg;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                bw[e] = static_cast<uint32_t>(bp[2 * e]) |
+                                        (static_cast<uint32_t>(bp[2 * e + 1]) << 16);
+                        }
+                    }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         float z0 = __uint_as_float(v[8 * g + 2 * e]);
                         float z1 = __uint_as_float(v[8 * g + 2 * e + 1]);
                         if constexpr (HAS_BIAS) {
-                            z0 += load16<IS_BF16>(p.bias, cg + 2 * e);
-                            z1 += load16<IS_BF16>(p.bias, cg + 2 * e + 1);
+                            z0 += unpack_lo<IS_BF16>(bw[e]);
+                            z1 += unpack_hi<IS_BF16>(bw[e]);
                         }
                         w[e] = pack2<IS_BF16>(activate<ACT>(z0), activate<ACT>(z1));
                     }

@@ -133,3 +133,25 @@ def test_both_tile_shapes(M, N, K, tiles):
     torch.cuda.synchronize()
     assert af.attn_fwd_status() == 0
     check(c, a, w, b, af.GEMM_ACT_GELU, "bf16", f"{M}x{N}x{K} tiles flag {tiles}")
+
+
+def test_bias_not_16_byte_aligned():
+    """A bias that starts 2 bytes past a 16-byte boundary takes the element-wise bias
+    loads; the result is the same."""
+    M, N, K = 300, 264, 200
+    a, w, b = make_gemm(M, N, K, "f16", seed=77)
+    da, dw = a.cuda(), w.cuda()
+    store = torch.zeros(N + 8, dtype=torch.float16, device="cuda")
+    store[1:N + 1] = b.cuda()
+    db = store[1:N + 1]
+    assert db.data_ptr() % 16 == 2
+    c = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    rc = af.gemm_bias_act_raw(da.data_ptr(), dw.data_ptr(), db.data_ptr(), c.data_ptr(), M, N,
+                              K, af.GEMM_ACT_GELU, af.ATTN_F16,
+                              torch.cuda.current_stream().cuda_stream)
+    assert rc == af.ATTN_OK
+    torch.cuda.synchronize()
+    check(c, a, w, b, af.GEMM_ACT_GELU, "f16", "unaligned bias")
+    c2 = af.gemm_bias_act(da, dw, b.cuda(), af.GEMM_ACT_GELU)
+    torch.cuda.synchronize()
+    assert torch.equal(c, c2)
