@@ -696,7 +696,9 @@ def main():
                 print(json.dumps(reference_arm(args, 1, rank)), flush=True)
             return
         line = cuda_arm(args, world, rank, local)
-        if rank == 0 and not args.no_extra:
+        # the other workloads once, on a single-GPU run (a multi-GPU run would hold every
+        # GPU while rank 0 alone works through them)
+        if rank == 0 and world == 1 and not args.no_extra:
             line["extra"] = extra_workloads(["C3", "C4", "C5"], world)
             line["extra"]["cuda_graph"] = graph_launches(["C1", "C2"])
             line["extra"]["decode_splitkv"] = decode_workloads(
