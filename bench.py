@@ -484,6 +484,47 @@ def decode_workloads(names):
     return res
 
 
+def prefill_workloads(names):
+    """Grouped K/V heads with the bottom-right causal mask (attn_fwd_ex, whole pass),
+    TFLOP/s at 4*D FLOPs per visible (query, key) pair."""
+    import attention_forward_18_b200 as af
+    from workloads import PREFILL_WORKLOADS, visible_pairs
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_kind = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    res = {}
+    for name in names:
+        w = PREFILL_WORKLOADS[name]
+        q, k, v = (t.to(dev) for t in make_inputs(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+        dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
+        mask = af.ATTN_MASK_CAUSAL_BOTTOM_RIGHT
+
+        def f():
+            rc = af.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), w.B, w.H, w.kv_heads, w.Sq, w.Sk, w.D, mask,
+                                w.scale, dcode, 0, None, 0, stream.cuda_stream)
+            if rc != 0:
+                raise af.AttnError(rc, "attn_fwd_ex")
+        ms = statistics.median(t[0] for t in time_steps([f], 20, 5, flush, stream))
+        flops = 4.0 * w.D * w.B * w.H * visible_pairs(w.Sq, w.Sk, 2)
+        tf = flops / (ms * 1e-3) / 1e12
+        res[name] = {"shape": f"B={w.B} H={w.H} Hkv={w.kv_heads} Sq={w.Sq} Sk={w.Sk} D={w.D} "
+                              f"{w.dtype} bottom-right causal",
+                     "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                     "frac_of_peak": round(tf / peak, 4)}
+        status = af.attn_fwd_status(stream)
+        if status != 0:
+            raise af.AttnError(status, f"device status after {name}")
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+    res["peak_TFLOP/s"] = f"{peak} ({peak_kind} dense bf16 burst)"
+    return res
+
+
 def softmax_workloads(names):
     """The standalone row softmax (HBM-bound: x read once, y written once), timed like
     the rest with a cold L2, as GB/s of those algorithmic bytes."""
@@ -703,6 +744,7 @@ def main():
             line["extra"]["cuda_graph"] = graph_launches(["C1", "C2"])
             line["extra"]["decode_splitkv"] = decode_workloads(
                 ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])
+            line["extra"]["prefill_grouped_bottom_right"] = prefill_workloads(["PRE1"])
             line["extra"]["row_softmax"] = softmax_workloads(["SMX1", "SMX2", "SMX3"])
             line["extra"]["gemm_bias_act"] = gemm_workloads(["GEMM1", "GEMM2", "GEMM3"])
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -107,3 +107,20 @@ def test_grouped_heads_equal_repeated_heads():
         torch.cuda.synchronize()
         assert (o1.float() - o2.float()).abs().max().item() <= O_TOL
         assert (l1 - l2).abs().max().item() <= LSE_TOL
+
+
+def test_prefill_workload_in_bench_configuration():
+    """The benchmark's chunked-prefill workload (grouped heads, bottom-right causal) at
+    full size: sampled rows against the oracle."""
+    from workloads import PREFILL_WORKLOADS, make_inputs, sample_rows
+    w = PREFILL_WORKLOADS["PRE1"]
+    q, k, v = make_inputs(w)
+    o, lse = af.attention_ex(q.cuda(), k.cuda(), v.cuda(), mask=af.ATTN_MASK_CAUSAL_BOTTOM_RIGHT,
+                             scale=w.scale)
+    torch.cuda.synchronize()
+    assert af.attn_fwd_status() == 0
+    rows = sample_rows(w.B, w.H, w.Sq, 48, seed=w.seed)
+    ro, rl = oracle.attn_ref_rows_ex(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                     rows, oracle.CAUSAL_BOTTOM_RIGHT, w.scale)
+    idx = tuple(np.array(rows).T)
+    compare_ex(o.double().cpu().numpy()[idx], lse.double().cpu().numpy()[idx], ro, rl, "PRE1")

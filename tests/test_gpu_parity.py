@@ -111,3 +111,33 @@ def test_host_buffers_entry_point():
     o_ref, l_ref = oracle.attn_ref(q.double().numpy(), k.double().numpy(), v.double().numpy(),
                                    True, 1 / np.sqrt(D))
     compare(oh.double().numpy(), lh.double().numpy(), o_ref, l_ref, "host entry")
+
+
+def test_concurrent_streams_do_not_interfere():
+    """The library keeps no per-call state on the device: four passes of different
+    shapes, masks and paths (whole, split, grouped heads) in flight at once on four
+    streams each match the oracle."""
+    cases = [
+        (dict(B=2, H=4, Sq=700, Sk=900, D=128, dtype="bf16", seed=91), af.ATTN_MASK_CAUSAL, 0, 4),
+        (dict(B=1, H=8, Sq=1, Sk=20000, D=64, dtype="f16", seed=92), af.ATTN_MASK_NONE, None, 8),
+        (dict(B=3, H=2, Sq=300, Sk=300, D=64, dtype="f16", seed=93), af.ATTN_MASK_NONE, 0, 2),
+        (dict(B=1, H=8, Sq=33, Sk=5000, D=128, dtype="bf16", seed=94),
+         af.ATTN_MASK_CAUSAL_BOTTOM_RIGHT, 3, 2),
+    ]
+    streams = [torch.cuda.Stream() for _ in cases]
+    runs = []
+    for (kw, mask, n_splits, Hkv), st in zip(cases, streams):
+        q, _, _ = make_qkv(kw["B"], kw["H"], kw["Sq"], 1, kw["D"], kw["dtype"], kw["seed"])
+        _, k, v = make_qkv(kw["B"], Hkv, 1, kw["Sk"], kw["D"], kw["dtype"], kw["seed"] + 1)
+        with torch.cuda.stream(st):
+            dq, dk, dv = (t.cuda(non_blocking=False) for t in (q, k, v))
+            o, lse = af.attention_ex(dq, dk, dv, mask=mask, scale=0.1, n_splits=n_splits,
+                                     stream=st)
+        runs.append((q, k, v, mask, o, lse))
+    torch.cuda.synchronize()
+    assert af.attn_fwd_status() == 0
+    for (q, k, v, mask, o, lse) in runs:
+        o_ref, lse_ref = oracle.attn_ref_ex(q.double().numpy(), k.double().numpy(),
+                                            v.double().numpy(), mask, 0.1)
+        compare(o.double().cpu().numpy(), lse.double().cpu().numpy(), o_ref, lse_ref,
+                f"stream case mask={mask}")

@@ -88,6 +88,28 @@ DECODE_WORKLOADS = {
 }
 
 
+# Chunked prefill with grouped K/V heads and the bottom-right causal mask: a chunk of
+# 2048 new query rows attends to the 8192 keys of its context (the 6144 before it and
+# itself, causally).
+PREFILL_WORKLOADS = {
+    "PRE1": Workload("PRE1", 1, 32, 2048, 8192, 128, "bf16", (True,), 10, Hkv=8,
+                     note="chunked prefill: 2048 new rows, 8192-key context, 32 query "
+                          "heads on 8 K/V heads, bottom-right causal"),
+}
+
+
+def visible_pairs(Sq, Sk, mask):
+    """Number of (query, key) pairs a mask lets through per head: 0 none, 1 top-left
+    causal (key j visible iff j <= i), 2 bottom-right (iff j <= i + Sk - Sq)."""
+    if mask == 0:
+        return Sq * Sk
+    off = 0 if mask == 1 else Sk - Sq
+    total = 0
+    for i in range(Sq):
+        total += max(0, min(Sk, i + off + 1))
+    return total
+
+
 @dataclass(frozen=True)
 class RowWorkload:
     """A rows x n matrix for the standalone row softmax: i.i.d. N(0, 1) times `scale`
