@@ -124,3 +124,22 @@ def test_prefill_workload_in_bench_configuration():
                                      rows, oracle.CAUSAL_BOTTOM_RIGHT, w.scale)
     idx = tuple(np.array(rows).T)
     compare_ex(o.double().cpu().numpy()[idx], lse.double().cpu().numpy()[idx], ro, rl, "PRE1")
+
+
+@pytest.mark.parametrize("scale", [-0.2, 0.0])
+@pytest.mark.parametrize("mask", ["none", "topleft", "bottomright"])
+@pytest.mark.parametrize("n_splits", [0, 3])
+def test_negative_and_zero_scale_on_every_path(n_splits, mask, scale):
+    """The negative-scale and zero-scale handling on the split, grouped-head, general
+    causal and decode instantiations (a decode shape: 4 packed rows per K/V head) and on
+    a longer prefill shape."""
+    for (Sq, Sk) in ((1, 2000), (300, 700)):
+        q, k, v = make_gqa(2, 8, 2, Sq, Sk, 64, "f16", seed=Sq + Sk)
+        dq, dk, dv = (t.cuda() for t in (q, k, v))
+        o, lse = af.attention_ex(dq, dk, dv, mask=MASKS[mask], scale=scale, n_splits=n_splits)
+        torch.cuda.synchronize()
+        assert af.attn_fwd_status() == 0
+        o_ref, lse_ref = oracle.attn_ref_ex(q.double().numpy(), k.double().numpy(),
+                                            v.double().numpy(), MASKS[mask], scale)
+        compare_ex(o.double().cpu().numpy(), lse.double().cpu().numpy(), o_ref, lse_ref,
+                   f"scale {scale} mask {mask} splits {n_splits} Sq {Sq}")
