@@ -117,6 +117,12 @@ int noalloc_scratch(void** out) {
     return ATTN_OK;
 }
 
+// Head dimensions: 64 and 128 run at their size; 80, 96 and 112 run in the D = 128
+// kernel with Q, K, V zero-padded by the TMA loads (columns past D read as zeros, so
+// the scores and the output are unchanged) and O written for D columns.
+bool head_dim_ok(int D) { return D == 64 || D == 80 || D == 96 || D == 112 || D == 128; }
+int kernel_d(int D) { return D <= 64 ? 64 : 128; }
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return x < y + nb && y < x + na;
@@ -127,7 +133,7 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
              int B, int H, int Hkv, int Sq, int Sk, int D, float scale, int dtype) {
     if (!q || !k || !v || !o) return ATTN_ERR_NULLPTR;
     if (dtype != ATTN_F16 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
-    if (D != 64 && D != 128) return ATTN_ERR_HEADDIM;
+    if (!head_dim_ok(D)) return ATTN_ERR_HEADDIM;
     if (B < 1 || H < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || H % Hkv != 0) return ATTN_ERR_SHAPE;
     if (Sq > kMaxSeq || Sk > kMaxSeq) return ATTN_ERR_SHAPE;
     const int64_t bh = static_cast<int64_t>(B) * H;
@@ -240,6 +246,9 @@ int launch_merge(const float* ws_o, const float* ws_lse, void* o, float* lse, in
     if (D == 64) {
         if (bf16) attn::attn_splitkv_merge_kernel<64, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
         else attn::attn_splitkv_merge_kernel<64, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+    } else if (D != 128) {
+        if (bf16) attn::attn_splitkv_merge_any_d<true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows, D);
+        else attn::attn_splitkv_merge_any_d<false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows, D);
     } else {
         if (bf16) attn::attn_splitkv_merge_kernel<128, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
         else attn::attn_splitkv_merge_kernel<128, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
@@ -295,6 +304,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     p.BH = BH;
     p.n_qp = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
     p.sq_head = Sq;
+    p.d_out = D;
     p.causal_off = mask == ATTN_MASK_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
     const int n_kv = (Sk + attn::BN - 1) / attn::BN;
     p.n_splits = n_splits > 0 ? n_splits : 1;
@@ -314,8 +324,8 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     if (n_units > INT_MAX) return ATTN_ERR_SHAPE;
     const int grid = n_units < num_sms ? static_cast<int>(n_units) : num_sms;
     const bool c = mask != ATTN_MASK_NONE;
-    if (n_splits == 0) return launch_any<false>(tq, tk, tv, p, grid, D, bf16, c, stream);
-    rc = launch_any<true>(tq, tk, tv, p, grid, D, bf16, c, stream);
+    if (n_splits == 0) return launch_any<false>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
+    rc = launch_any<true>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
     if (rc != ATTN_OK) return rc;
     return launch_merge(p.ws_o, p.ws_lse, o, lse, n_splits, static_cast<int64_t>(B) * H * Sq, D,
                         bf16, stream);
@@ -396,7 +406,7 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
 }
 
 size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_splits) {
-    if (B < 1 || H < 1 || Sq < 1 || (D != 64 && D != 128) || n_splits < 1 ||
+    if (B < 1 || H < 1 || Sq < 1 || !head_dim_ok(D) || n_splits < 1 ||
         n_splits > kMaxSplits)
         return 0;
     return ws_bytes(B, H, Sq, D, n_splits);
@@ -476,7 +486,7 @@ const char* attn_fwd_strerror(int code) {
         case ATTN_ERR_NULLPTR: return "null pointer argument";
         case ATTN_ERR_ALIGN: return "misaligned pointer (q/k/v/o need 16 bytes, lse 4)";
         case ATTN_ERR_SHAPE: return "bad shape (B, H, Sq, Sk >= 1 and within limits)";
-        case ATTN_ERR_HEADDIM: return "unsupported head dimension (64 or 128)";
+        case ATTN_ERR_HEADDIM: return "unsupported head dimension (64, 80, 96, 112 or 128)";
         case ATTN_ERR_DTYPE: return "unsupported dtype (ATTN_F16 or ATTN_BF16)";
         case ATTN_ERR_TENSORMAP: return "TMA descriptor encoding failed";
         case ATTN_ERR_LAUNCH: return "CUDA call or kernel launch failed";

@@ -84,6 +84,8 @@ struct Params {
     float* ws_lse;      // split-KV: [n_splits, BH, Sq] fp32 partial LSE
     int Sq, Sk, BH, n_qp;  // packed query rows, keys, K/V heads, 256-row query pairs
     int sq_head;        // query positions per query head (Sq / g)
+    int d_out;          // head dimension of the tensors (<= D; Q, K, V read as zero-padded
+                        // to D, O and the partials written for d_out columns)
     int causal_off;     // causal: key j visible to position i iff j <= i + causal_off
     int n_splits;       // KV ranges per (query pair, head); 1 for the whole pass
     int chunk_tiles;    // KV tiles per range
@@ -343,15 +345,15 @@ template <int D, bool SPLIT>
 __device__ __forceinline__ void write_empty_row(const Params& p, int64_t head_row, int bh,
                                                 int qrow) {
     if constexpr (SPLIT) {
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D);
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * p.d_out);
 #pragma unroll 1
-        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < p.d_out / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         p.ws_lse[head_row * p.Sq + qrow] = -INFINITY;
     } else {
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
-                                              (static_cast<int64_t>(bh) * p.Sq + qrow) * D);
+                                              (static_cast<int64_t>(bh) * p.Sq + qrow) * p.d_out);
 #pragma unroll 1
-        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < p.d_out / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
         if (p.lse != nullptr) p.lse[static_cast<int64_t>(bh) * p.Sq + qrow] = -INFINITY;
     }
 }
@@ -362,11 +364,11 @@ template <int D, bool IS_BF16, bool SPLIT>
 __device__ __forceinline__ void store_o8(const Params& p, int64_t head_row, int bh, int qrow,
                                          int c, const float (&f)[8]) {
     if constexpr (SPLIT) {
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D + 8 * c);
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * p.d_out + 8 * c);
         dst[0] = make_float4(f[0], f[1], f[2], f[3]);
         dst[1] = make_float4(f[4], f[5], f[6], f[7]);
     } else {
-        uint16_t* o = reinterpret_cast<uint16_t*>(p.o) + (static_cast<int64_t>(bh) * p.Sq + qrow) * D;
+        uint16_t* o = reinterpret_cast<uint16_t*>(p.o) + (static_cast<int64_t>(bh) * p.Sq + qrow) * p.d_out;
         *reinterpret_cast<uint4*>(o + 8 * c) =
             make_uint4(pack2<IS_BF16>(f[0], f[1]), pack2<IS_BF16>(f[2], f[3]),
                        pack2<IS_BF16>(f[4], f[5]), pack2<IS_BF16>(f[6], f[7]));
@@ -572,7 +574,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     lt > 0.f ? (mx + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
                 const uint32_t tO0 = tmem + lane_base + TMEM_O;
 #pragma unroll 1
-                for (int c = 0; c < D / 8; ++c) {
+                for (int c = 0; c < p.d_out / 8; ++c) {
                     uint32_t o0[8], o1[8];
                     ptx::tmem_ld8(tO0 + 8 * c, o0);
                     if (nt1 > 0) ptx::tmem_ld8(tO0 + D + 8 * c, o1);
@@ -608,18 +610,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (w.n[t] == 0) {
                     // no key of the unit's range is visible to these rows: O = 0 and
                     // LSE = -inf (the empty sum)
-                    if (SPLIT && store) {
-                        float4* dst = reinterpret_cast<float4*>(p.ws_o + (head_row * p.Sq + qrow) * D);
-#pragma unroll 1
-                        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        p.ws_lse[head_row * p.Sq + qrow] = -INFINITY;
-                    } else if (!SPLIT && store) {
-                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
-                                                              (static_cast<int64_t>(w.bh) * p.Sq + qrow) * D);
-#pragma unroll 1
-                        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-                        if (p.lse != nullptr) p.lse[static_cast<int64_t>(w.bh) * p.Sq + qrow] = -INFINITY;
-                    }
+                    if (store) write_empty_row<D, SPLIT>(p, head_row, w.bh, qrow);
                     continue;
                 }
                 if (!(ok = warp_wait(ctx, B_ST(t), ut[t] & 1))) break;
@@ -634,9 +625,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
                 if constexpr (SPLIT) {
                     // partial O / l and LSE of this KV range, fp32
-                    float* orow = p.ws_o + (head_row * p.Sq + qrow) * D;
+                    float* orow = p.ws_o + (head_row * p.Sq + qrow) * p.d_out;
 #pragma unroll 1
-                    for (int c = 0; c < D / 16; ++c) {
+                    for (int c = 0; c < p.d_out / 16; ++c) {
                         uint32_t ov[16];
                         ptx::tmem_ld16(tO + 16 * c, ov);
                         ptx::tmem_wait_ld();
@@ -654,9 +645,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 } else {
                     // O / l in fp32, one rounding to 16 bits; LSE in natural log
                     uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) +
-                                     (static_cast<int64_t>(w.bh) * p.Sq + qrow) * D;
+                                     (static_cast<int64_t>(w.bh) * p.Sq + qrow) * p.d_out;
 #pragma unroll 1
-                    for (int c = 0; c < D / 16; ++c) {
+                    for (int c = 0; c < p.d_out / 16; ++c) {
                         uint32_t ov[16];
                         ptx::tmem_ld16(tO + 16 * c, ov);
                         ptx::tmem_wait_ld();

@@ -72,4 +72,42 @@ __global__ void __launch_bounds__(256)
     if (lane == 0 && lse != nullptr) lse[row] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
 }
 
+// The same merge for any head dimension d <= 128 (rows of d values): lane l takes
+// columns l, l + 32, l + 64, l + 96 (coalesced across the warp).
+template <bool IS_BF16>
+__global__ void __launch_bounds__(256)
+    attn_splitkv_merge_any_d(const float* __restrict__ ws_o, const float* __restrict__ ws_lse,
+                             void* __restrict__ o, float* __restrict__ lse, int n_splits,
+                             int64_t rows, int d) {
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float mx = -INFINITY;
+    for (int s = lane; s < n_splits; s += 32) mx = fmaxf(mx, ws_lse[s * rows + row]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float wsum = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+        const float ls = ws_lse[s * rows + row];
+        const float wgt = (ls == -INFINITY) ? 0.f : expf(ls - mx);
+        wsum += wgt;
+        const float* src = ws_o + (s * rows + row) * d;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (lane + 32 * i < d) acc[i] += wgt * src[lane + 32 * i];
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(o) + row * d;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (lane + 32 * i < d) {
+            const uint32_t pk = IS_BF16 ? ptx::pack_bf16x2(acc[i] * inv, 0.f)
+                                        : ptx::pack_f16x2(acc[i] * inv, 0.f);
+            dst[lane + 32 * i] = static_cast<uint16_t>(pk & 0xffffu);
+        }
+    }
+    if (lane == 0 && lse != nullptr) lse[row] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+}
+
 }  // namespace attn

@@ -55,7 +55,7 @@ def call(q=Q, k=K, v=V, o=O, lse=L, B=1, H=2, Sq=128, Sk=128, D=64, causal=0,
     (dict(o=None), af.ATTN_ERR_NULLPTR),
     (dict(dtype=2), af.ATTN_ERR_DTYPE),
     (dict(dtype=-1), af.ATTN_ERR_DTYPE),
-    (dict(D=96), af.ATTN_ERR_HEADDIM),
+    (dict(D=72), af.ATTN_ERR_HEADDIM),
     (dict(D=0), af.ATTN_ERR_HEADDIM),
     (dict(B=0), af.ATTN_ERR_SHAPE),
     (dict(H=-1), af.ATTN_ERR_SHAPE),
@@ -124,7 +124,10 @@ def test_splitkv_workspace_size_formula():
     B, H, Sq, D, S = 2, 3, 17, 64, 5
     o_part = -(-(S * B * H * Sq * D * 4) // 256) * 256
     assert af.splitkv_workspace_bytes(B, H, Sq, D, S) == o_part + S * B * H * Sq * 4
-    assert af.splitkv_workspace_bytes(B, H, Sq, 96, S) == 0
+    assert af.splitkv_workspace_bytes(B, H, Sq, 72, S) == 0
+    # head dimensions run zero-padded in the D = 128 kernel keep their own row size
+    assert af.splitkv_workspace_bytes(B, H, Sq, 96, S) == (
+        -(-(S * B * H * Sq * 96 * 4) // 256) * 256 + S * B * H * Sq * 4)
     assert af.splitkv_workspace_bytes(B, H, Sq, D, 0) == 0
     assert af.splitkv_workspace_bytes(B, H, Sq, D, 1025) == 0
 
@@ -151,7 +154,7 @@ def test_splitkv_default_splits_in_range():
     (dict(ws_bytes=1024), af.ATTN_ERR_WORKSPACE),
     (dict(ws=Q + 4096), af.ATTN_ERR_ALIAS),
     (dict(ws=O - 256), af.ATTN_ERR_ALIAS),
-    (dict(D=80), af.ATTN_ERR_HEADDIM),
+    (dict(D=144), af.ATTN_ERR_HEADDIM),
 ])
 def test_splitkv_argument_errors(kw, code):
     assert split_call(**kw) == code
@@ -175,7 +178,7 @@ def ex_call(**kw):
     (dict(H=64, H_kv=1, Sq=1 << 19), af.ATTN_ERR_SHAPE),   # 2^25 packed rows
     (dict(n_splits=-1), af.ATTN_ERR_SHAPE),
     (dict(n_splits=2), af.ATTN_ERR_NULLPTR),    # split pass without a workspace
-    (dict(D=96), af.ATTN_ERR_HEADDIM),
+    (dict(D=48), af.ATTN_ERR_HEADDIM),
     (dict(o=K + 4096), af.ATTN_ERR_ALIAS),      # inside K (sized with H_kv heads)
 ])
 def test_ex_argument_errors(kw, code):

@@ -143,3 +143,22 @@ def test_negative_and_zero_scale_on_every_path(n_splits, mask, scale):
                                             v.double().numpy(), MASKS[mask], scale)
         compare_ex(o.double().cpu().numpy(), lse.double().cpu().numpy(), o_ref, lse_ref,
                    f"scale {scale} mask {mask} splits {n_splits} Sq {Sq}")
+
+
+@pytest.mark.parametrize("D", [80, 96, 112])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("case", ["whole_nc", "whole_causal", "split_decode", "gqa_br",
+                                  "ragged"])
+def test_padded_head_dims(case, dtype, D):
+    """Head dimensions 80, 96 and 112 run in the D = 128 kernel with the missing
+    columns read as zeros; every path against the oracle."""
+    if case == "whole_nc":
+        check(2, 3, 3, 300, 500, D, dtype, "none", 0, seed=D)
+    elif case == "whole_causal":
+        check(2, 3, 3, 500, 500, D, dtype, "topleft", 0, seed=D + 1)
+    elif case == "split_decode":
+        check(2, 4, 4, 1, 5000, D, dtype, "none", None, seed=D + 2)
+    elif case == "gqa_br":
+        check(1, 8, 2, 40, 3000, D, dtype, "bottomright", 5, seed=D + 3)
+    else:
+        check(1, 2, 2, 129, 257, D, dtype, "none", 0, seed=D + 4)
