@@ -11,6 +11,7 @@
 
 #include "attn_fwd.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_fwd_wide_kernel.cuh"
 #include "attn_merge.cuh"
 
 // Library-owned scratch of attn_fwd_splitkv_noalloc: one copy per device, in the
@@ -49,8 +50,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // [BH, S, D] 16-bit tensor seen as 3-D (D innermost); box = 64 elements (128 bytes,
-// the swizzle span) x 128 rows x 1 head; rows past S read as zeros.
-bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool bf16) {
+// the swizzle span) x box_rows rows x 1 head; rows past S and columns past D read as
+// zeros.
+bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool bf16,
+                    int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
@@ -58,7 +61,7 @@ bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                    static_cast<cuuint64_t>(S) * D * 2};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(attn::CHUNK_ELEMS),
-                               static_cast<cuuint32_t>(attn::BN), 1};
+                               static_cast<cuuint32_t>(box_rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r =
         fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
@@ -119,9 +122,16 @@ int noalloc_scratch(void** out) {
 
 // Head dimensions: 64 and 128 run at their size; 80, 96 and 112 run in the D = 128
 // kernel with Q, K, V zero-padded by the TMA loads (columns past D read as zeros, so
-// the scores and the output are unchanged) and O written for D columns.
-bool head_dim_ok(int D) { return D == 64 || D == 80 || D == 96 || D == 112 || D == 128; }
-int kernel_d(int D) { return D <= 64 ? 64 : 128; }
+// the scores and the output are unchanged) and O written for D columns.  192 and 256
+// run in the wide kernel (one 128-row query tile per CTA, 64-key KV tiles).
+bool head_dim_ok(int D) {
+    return D == 64 || D == 80 || D == 96 || D == 112 || D == 128 || D == 192 || D == 256;
+}
+int kernel_d(int D) { return D <= 64 ? 64 : D <= 128 ? 128 : D; }
+bool is_wide(int D) { return D > 128; }
+// query rows and keys per work unit and KV tile of the kernel that runs D
+int unit_rows(int D) { return is_wide(D) ? attn::wide::WBM : attn::ROWS_PER_CTA; }
+int kv_tile_keys(int D) { return is_wide(D) ? attn::wide::WBN : attn::BN; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -141,7 +151,7 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     // the kernel's rows: g = H / Hkv query heads packed per K/V head
     const int64_t rows = static_cast<int64_t>(H / Hkv) * Sq;
     if (rows > kMaxSeq) return ATTN_ERR_SHAPE;
-    const int64_t n_qp = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    const int64_t n_qp = (rows + unit_rows(D) - 1) / unit_rows(D);
     if (n_qp * B * Hkv > INT_MAX) return ATTN_ERR_SHAPE;
     if (!std::isfinite(scale)) return ATTN_ERR_SCALE;
     auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
@@ -229,6 +239,59 @@ int launch_any(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                 : launch_d<128, false, SPLIT>(tq, tk, tv, p, grid, causal, s);
 }
 
+template <int D, int NS, bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
+int launch_wide_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const attn::Params& p, int grid, cudaStream_t stream) {
+    auto kern = attn::wide::attn_fwd_wide_kernel<D, NS, BF16, CAUSAL, NEG, SPLIT, GEN>;
+    constexpr int smem = attn::wide::Layout<D, NS>::ALLOC;
+    static bool attr_set[kMaxDevices];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_LAUNCH;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            attr_set[dev] = true;
+        }
+    }
+    kern<<<grid, attn::wide::NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+// Wide kernel ring depth: 64-key K/V stages beside the 128-row Q tile (~192 KB).
+template <int D>
+constexpr int kWideStages = (D == 256) ? 2 : 3;
+
+template <int D, bool BF16, bool SPLIT>
+int launch_wide_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                  const attn::Params& p, int grid, bool causal, cudaStream_t s) {
+    constexpr int NS = kWideStages<D>;
+    const bool neg = p.scale_log2 < 0.f;
+    if (causal && (p.causal_off != 0 || p.sq_head != p.Sq))
+        return neg ? launch_wide_one<D, NS, BF16, true, true, SPLIT, true>(tq, tk, tv, p, grid, s)
+                   : launch_wide_one<D, NS, BF16, true, false, SPLIT, true>(tq, tk, tv, p, grid, s);
+    if (causal)
+        return neg ? launch_wide_one<D, NS, BF16, true, true, SPLIT, false>(tq, tk, tv, p, grid, s)
+                   : launch_wide_one<D, NS, BF16, true, false, SPLIT, false>(tq, tk, tv, p, grid, s);
+    return neg ? launch_wide_one<D, NS, BF16, false, true, SPLIT, false>(tq, tk, tv, p, grid, s)
+               : launch_wide_one<D, NS, BF16, false, false, SPLIT, false>(tq, tk, tv, p, grid, s);
+}
+
+template <bool SPLIT>
+int launch_wide(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const attn::Params& p, int grid, int D, bool bf16, bool causal,
+                cudaStream_t s) {
+    if (D == 192) return bf16 ? launch_wide_d<192, true, SPLIT>(tq, tk, tv, p, grid, causal, s)
+                              : launch_wide_d<192, false, SPLIT>(tq, tk, tv, p, grid, causal, s);
+    return bf16 ? launch_wide_d<256, true, SPLIT>(tq, tk, tv, p, grid, causal, s)
+                : launch_wide_d<256, false, SPLIT>(tq, tk, tv, p, grid, causal, s);
+}
+
 // Workspace of a split pass: partial O [n_splits, B*H, Sq, D] fp32, then partial LSE
 // [n_splits, B*H, Sq] fp32 at the next 256-byte boundary.
 size_t ws_o_bytes(int B, int H, int Sq, int D, int n_splits) {
@@ -246,6 +309,12 @@ int launch_merge(const float* ws_o, const float* ws_lse, void* o, float* lse, in
     if (D == 64) {
         if (bf16) attn::attn_splitkv_merge_kernel<64, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
         else attn::attn_splitkv_merge_kernel<64, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+    } else if (D == 192) {
+        if (bf16) attn::attn_splitkv_merge_kernel<192, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+        else attn::attn_splitkv_merge_kernel<192, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+    } else if (D == 256) {
+        if (bf16) attn::attn_splitkv_merge_kernel<256, true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
+        else attn::attn_splitkv_merge_kernel<256, false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows);
     } else if (D != 128) {
         if (bf16) attn::attn_splitkv_merge_any_d<true><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows, D);
         else attn::attn_splitkv_merge_any_d<false><<<blocks, 256, 0, s>>>(ws_o, ws_lse, o, lse, n_splits, rows, D);
@@ -291,9 +360,12 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int BH = B * Hkv;
     const int rows = (H / Hkv) * Sq;
     const bool bf16 = dtype == ATTN_BF16;
+    const bool wide = is_wide(D);
+    const int kv_keys = kv_tile_keys(D);
     CUtensorMap tq, tk, tv;
-    if (!encode_qkv_map(&tq, q, D, rows, BH, bf16) || !encode_qkv_map(&tk, k, D, Sk, BH, bf16) ||
-        !encode_qkv_map(&tv, v, D, Sk, BH, bf16))
+    if (!encode_qkv_map(&tq, q, D, rows, BH, bf16, attn::BM) ||
+        !encode_qkv_map(&tk, k, D, Sk, BH, bf16, kv_keys) ||
+        !encode_qkv_map(&tv, v, D, Sk, BH, bf16, kv_keys))
         return ATTN_ERR_TENSORMAP;
 
     attn::Params p;
@@ -302,11 +374,11 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     p.Sq = rows;
     p.Sk = Sk;
     p.BH = BH;
-    p.n_qp = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA;
+    p.n_qp = (rows + unit_rows(D) - 1) / unit_rows(D);  // query units (wide: tiles)
     p.sq_head = Sq;
     p.d_out = D;
     p.causal_off = mask == ATTN_MASK_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
-    const int n_kv = (Sk + attn::BN - 1) / attn::BN;
+    const int n_kv = (Sk + kv_keys - 1) / kv_keys;
     p.n_splits = n_splits > 0 ? n_splits : 1;
     p.chunk_tiles = (n_kv + p.n_splits - 1) / p.n_splits;
     p.ws_o = n_splits > 0 ? static_cast<float*>(workspace) : nullptr;
@@ -324,8 +396,11 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     if (n_units > INT_MAX) return ATTN_ERR_SHAPE;
     const int grid = n_units < num_sms ? static_cast<int>(n_units) : num_sms;
     const bool c = mask != ATTN_MASK_NONE;
-    if (n_splits == 0) return launch_any<false>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
-    rc = launch_any<true>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
+    if (n_splits == 0)
+        return wide ? launch_wide<false>(tq, tk, tv, p, grid, D, bf16, c, stream)
+                    : launch_any<false>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
+    rc = wide ? launch_wide<true>(tq, tk, tv, p, grid, D, bf16, c, stream)
+              : launch_any<true>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
     if (rc != ATTN_OK) return rc;
     return launch_merge(p.ws_o, p.ws_lse, o, lse, n_splits, static_cast<int64_t>(B) * H * Sq, D,
                         bf16, stream);
@@ -486,7 +561,7 @@ const char* attn_fwd_strerror(int code) {
         case ATTN_ERR_NULLPTR: return "null pointer argument";
         case ATTN_ERR_ALIGN: return "misaligned pointer (q/k/v/o need 16 bytes, lse 4)";
         case ATTN_ERR_SHAPE: return "bad shape (B, H, Sq, Sk >= 1 and within limits)";
-        case ATTN_ERR_HEADDIM: return "unsupported head dimension (64, 80, 96, 112 or 128)";
+        case ATTN_ERR_HEADDIM: return "unsupported head dimension (64, 80, 96, 112, 128, 192 or 256)";
         case ATTN_ERR_DTYPE: return "unsupported dtype (ATTN_F16 or ATTN_BF16)";
         case ATTN_ERR_TENSORMAP: return "TMA descriptor encoding failed";
         case ATTN_ERR_LAUNCH: return "CUDA call or kernel launch failed";

@@ -43,16 +43,22 @@ __global__ void __launch_bounds__(256)
         const float wgt = (ls == -INFINITY) ? 0.f : expf(ls - mx);
         wsum += wgt;
         const float* src = ws_o + (s * rows + row) * D + lane * V;
-        if constexpr (V == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(src);
-            acc[0] += wgt * x.x;
-            acc[1] += wgt * x.y;
-            acc[2] += wgt * x.z;
-            acc[3] += wgt * x.w;
+        if constexpr (V % 4 == 0) {
+#pragma unroll
+            for (int e = 0; e < V; e += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(src + e);
+                acc[e] += wgt * x.x;
+                acc[e + 1] += wgt * x.y;
+                acc[e + 2] += wgt * x.z;
+                acc[e + 3] += wgt * x.w;
+            }
         } else {
-            const float2 x = *reinterpret_cast<const float2*>(src);
-            acc[0] += wgt * x.x;
-            acc[1] += wgt * x.y;
+#pragma unroll
+            for (int e = 0; e < V; e += 2) {
+                const float2 x = *reinterpret_cast<const float2*>(src + e);
+                acc[e] += wgt * x.x;
+                acc[e + 1] += wgt * x.y;
+            }
         }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -65,10 +71,14 @@ __global__ void __launch_bounds__(256)
             packed[e] = ptx::pack_f16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
     }
     uint16_t* dst = reinterpret_cast<uint16_t*>(o) + row * D + lane * V;
-    if constexpr (V == 4)
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    else
-        *reinterpret_cast<uint32_t*>(dst) = packed[0];
+    if constexpr (V % 4 == 0) {
+#pragma unroll
+        for (int e = 0; e < V / 2; e += 2)
+            *reinterpret_cast<uint2*>(dst + 2 * e) = make_uint2(packed[e], packed[e + 1]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < V / 2; ++e) *reinterpret_cast<uint32_t*>(dst + 2 * e) = packed[e];
+    }
     if (lane == 0 && lse != nullptr) lse[row] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
 }
 

@@ -348,9 +348,10 @@ def extra_workloads(af_names, world):
     flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     peaks, peak_kind = measured_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    from workloads import WIDE_WORKLOADS
     res = {}
     for name in af_names:
-        w = WORKLOADS[name]
+        w = WORKLOADS[name] if name in WORKLOADS else WIDE_WORKLOADS[name]
         q, k, v = (t.to(dev) for t in make_inputs(w))
         o = torch.empty_like(q)
         lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
@@ -693,9 +694,18 @@ def profile_extra(spec):
     along its first dimension so an ncu capture stays small)."""
     import dataclasses
     import attention_forward_18_b200 as af
-    from workloads import DECODE_WORKLOADS, GEMM_WORKLOADS, SOFTMAX_WORKLOADS, make_gemm, make_rows
+    from workloads import (DECODE_WORKLOADS, GEMM_WORKLOADS, SOFTMAX_WORKLOADS, WIDE_WORKLOADS,
+                           make_gemm, make_rows)
     name, _, cut = spec.partition(":")
-    if name in DECODE_WORKLOADS:
+    if name in WIDE_WORKLOADS:
+        w = WIDE_WORKLOADS[name]
+        if cut:
+            w = dataclasses.replace(w, H=int(cut))
+        q, k, v = (t.cuda() for t in make_inputs(w))
+        for c in w.causal:
+            af.attention(q, k, v, causal=c, scale=w.scale)
+        shape = f"B={w.B} H={w.H} S={w.Sq} D={w.D} causal={list(w.causal)}"
+    elif name in DECODE_WORKLOADS:
         w = DECODE_WORKLOADS[name]
         if cut:
             w = dataclasses.replace(w, B=int(cut))
@@ -740,7 +750,7 @@ def main():
         # the other workloads once, on a single-GPU run (a multi-GPU run would hold every
         # GPU while rank 0 alone works through them)
         if rank == 0 and world == 1 and not args.no_extra:
-            line["extra"] = extra_workloads(["C3", "C4", "C5"], world)
+            line["extra"] = extra_workloads(["C3", "C4", "C5", "WD192", "WD256"], world)
             line["extra"]["cuda_graph"] = graph_launches(["C1", "C2"])
             line["extra"]["decode_splitkv"] = decode_workloads(
                 ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])

@@ -59,7 +59,7 @@ enum {
     ATTN_ERR_NULLPTR = -1,   /* q, k, v or o is null                                */
     ATTN_ERR_ALIGN = -2,     /* q, k, v, o not 16-byte aligned, or lse not 4-byte   */
     ATTN_ERR_SHAPE = -3,     /* B, H, Sq or Sk < 1, or a size beyond the limits     */
-    ATTN_ERR_HEADDIM = -4,   /* D is not 64, 80, 96, 112 or 128                     */
+    ATTN_ERR_HEADDIM = -4,   /* D is not 64, 80, 96, 112, 128, 192 or 256           */
     ATTN_ERR_DTYPE = -5,     /* dtype is not ATTN_F16 / ATTN_BF16                   */
     ATTN_ERR_TENSORMAP = -6, /* the driver refused a TMA descriptor                 */
     ATTN_ERR_LAUNCH = -7,    /* a CUDA call or the kernel launch failed             */
@@ -77,9 +77,10 @@ enum {
  *   k, v   device, [B,H,Sk,D] 16-bit, 16-byte aligned
  *   o      device, [B,H,Sq,D] 16-bit, 16-byte aligned, written; must not overlap q/k/v
  *   lse    device, [B,H,Sq] fp32, written; may be NULL (not written)
- *   B, H, Sq, Sk >= 1; B*H, Sq, Sk <= 2^24; D in {64, 80, 96, 112, 128} (80, 96 and
- *          112 run as 128 with the missing columns read as zeros: exact, at the cost of
- *          the padded work)
+ *   B, H, Sq, Sk >= 1; B*H, Sq, Sk <= 2^24; D in {64, 80, 96, 112, 128, 192, 256}
+ *          (80, 96 and 112 run as 128 with the missing columns read as zeros: exact, at
+ *          the cost of the padded work; 192 and 256 run in a kernel of their own with
+ *          128-row query tiles and 64-key K/V tiles)
  *   causal 0: every key visible; nonzero: key j visible to query i iff j <= i
  *   scale  finite multiplier of q.k (e.g. 1/sqrt(D)); |scale*q.k| must fit fp32
  *   dtype  ATTN_F16 or ATTN_BF16

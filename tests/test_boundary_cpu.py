@@ -57,6 +57,9 @@ def call(q=Q, k=K, v=V, o=O, lse=L, B=1, H=2, Sq=128, Sk=128, D=64, causal=0,
     (dict(dtype=-1), af.ATTN_ERR_DTYPE),
     (dict(D=72), af.ATTN_ERR_HEADDIM),
     (dict(D=0), af.ATTN_ERR_HEADDIM),
+    (dict(D=160), af.ATTN_ERR_HEADDIM),
+    (dict(D=224), af.ATTN_ERR_HEADDIM),
+    (dict(D=320), af.ATTN_ERR_HEADDIM),
     (dict(B=0), af.ATTN_ERR_SHAPE),
     (dict(H=-1), af.ATTN_ERR_SHAPE),
     (dict(Sq=0), af.ATTN_ERR_SHAPE),
@@ -128,6 +131,11 @@ def test_splitkv_workspace_size_formula():
     # head dimensions run zero-padded in the D = 128 kernel keep their own row size
     assert af.splitkv_workspace_bytes(B, H, Sq, 96, S) == (
         -(-(S * B * H * Sq * 96 * 4) // 256) * 256 + S * B * H * Sq * 4)
+    # and so do the wide head dimensions
+    for Dw in (192, 256):
+        assert af.splitkv_workspace_bytes(B, H, Sq, Dw, S) == (
+            -(-(S * B * H * Sq * Dw * 4) // 256) * 256 + S * B * H * Sq * 4)
+    assert af.splitkv_workspace_bytes(B, H, Sq, 512, S) == 0
     assert af.splitkv_workspace_bytes(B, H, Sq, D, 0) == 0
     assert af.splitkv_workspace_bytes(B, H, Sq, D, 1025) == 0
 
@@ -179,6 +187,8 @@ def ex_call(**kw):
     (dict(n_splits=-1), af.ATTN_ERR_SHAPE),
     (dict(n_splits=2), af.ATTN_ERR_NULLPTR),    # split pass without a workspace
     (dict(D=48), af.ATTN_ERR_HEADDIM),
+    (dict(D=255), af.ATTN_ERR_HEADDIM),
+    (dict(D=256, H=64, H_kv=1, Sq=1 << 19), af.ATTN_ERR_SHAPE),  # wide kernel, 2^25 rows
     (dict(o=K + 4096), af.ATTN_ERR_ALIAS),      # inside K (sized with H_kv heads)
 ])
 def test_ex_argument_errors(kw, code):

@@ -88,6 +88,16 @@ DECODE_WORKLOADS = {
 }
 
 
+# Wide head dimensions (the wide kernel: one 128-row query tile per CTA, 64-key KV
+# tiles), non-causal and causal on the same tensors, same input recipe.
+WIDE_WORKLOADS = {
+    "WD192": Workload("WD192", 2, 16, 4096, 4096, 192, "bf16", (False, True), 30,
+                      note="head dimension 192"),
+    "WD256": Workload("WD256", 2, 16, 4096, 4096, 256, "bf16", (False, True), 31,
+                      note="head dimension 256"),
+}
+
+
 # Chunked prefill with grouped K/V heads and the bottom-right causal mask: a chunk of
 # 2048 new query rows attends to the 8192 keys of its context (the 6144 before it and
 # itself, causally).
