@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, f) for f in ("attn_fwd.cu", "row_softmax.cu", "gemm_bias_act.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("attn_fwd_kernel.cuh", "attn_fwd_wide_kernel.cuh", "attn_merge.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("attn_fwd_kernel.cuh", "attn_fwd_wide_kernel.cuh", "attn_fwd_pair_kernel.cuh", "attn_merge.cuh", "ptx.cuh")] + [
     os.path.join(ROOT, "include", h) for h in ("attn_fwd.h", "row_softmax.h", "gemm_bias_act.h")]
 LIB = os.path.join(HERE, "libattn_fwd.so")
 

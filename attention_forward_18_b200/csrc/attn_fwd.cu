@@ -12,6 +12,7 @@
 #include "attn_fwd.h"
 #include "attn_fwd_kernel.cuh"
 #include "attn_fwd_wide_kernel.cuh"
+#include "attn_fwd_pair_kernel.cuh"
 #include "attn_merge.cuh"
 
 // Library-owned scratch of attn_fwd_splitkv_noalloc: one copy per device, in the
@@ -65,6 +66,33 @@ bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r =
         fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The same tensor seen as 4-D (64 columns, S rows, D/64 column chunks, BH heads): a box
+// of 64 columns x box_rows rows x box_chunks chunks lands in shared memory chunk-major,
+// each chunk box_rows x 128 bytes in the 128-byte swizzle, as box_chunks 3-D boxes
+// would.  D a multiple of 64.
+bool encode_chunked_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool bf16,
+                        int box_rows, int box_chunks) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(attn::CHUNK_ELEMS),
+                                static_cast<cuuint64_t>(S),
+                                static_cast<cuuint64_t>(D / attn::CHUNK_ELEMS),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(attn::CHUNK_ELEMS) * 2,
+                                   static_cast<cuuint64_t>(S) * D * 2};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(attn::CHUNK_ELEMS),
+                               static_cast<cuuint32_t>(box_rows),
+                               static_cast<cuuint32_t>(box_chunks), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r =
+        fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -131,7 +159,6 @@ int kernel_d(int D) { return D <= 64 ? 64 : D <= 128 ? 128 : D; }
 bool is_wide(int D) { return D > 128; }
 // query rows and keys per work unit and KV tile of the kernel that runs D
 int unit_rows(int D) { return is_wide(D) ? attn::wide::WBM : attn::ROWS_PER_CTA; }
-int kv_tile_keys(int D) { return is_wide(D) ? attn::wide::WBN : attn::BN; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -263,6 +290,61 @@ int launch_wide_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
+// D = 256 on CTA pairs: clusters of two CTAs, the grid sized to the clusters that can
+// be resident at once (a persistent grid; the pair walks its units).
+template <bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
+int launch_pair_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const attn::Params& p, int64_t n_units, cudaStream_t stream) {
+    constexpr int NSK = 3, NSV = 2;  // K / V ring stages (224 KB with Q)
+    auto kern = attn::pair::attn_fwd_pair_kernel<NSK, NSV, BF16, CAUSAL, NEG, SPLIT, GEN>;
+    constexpr int smem = attn::pair::Layout<NSK, NSV>::ALLOC;
+    static int max_clusters[kMaxDevices];  // 0: not yet known
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_LAUNCH;
+    int clusters = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (max_clusters[dev] == 0) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            int sms = 0;
+            if (check_device(&sms) != ATTN_OK) return ATTN_ERR_DEVICE;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(sms - sms % 2), 1, 1);
+            cfg.blockDim = dim3(attn::pair::NUM_THREADS, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                return ATTN_ERR_LAUNCH;
+            }
+            max_clusters[dev] = n;
+        }
+        clusters = max_clusters[dev];
+    }
+    if (n_units < clusters) clusters = static_cast<int>(n_units);
+    kern<<<2 * clusters, attn::pair::NUM_THREADS, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
+}
+
+template <bool BF16, bool SPLIT>
+int launch_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const attn::Params& p, int64_t n_units, bool causal, cudaStream_t s) {
+    const bool neg = p.scale_log2 < 0.f;
+    if (causal && (p.causal_off != 0 || p.sq_head != p.Sq))
+        return neg ? launch_pair_one<BF16, true, true, SPLIT, true>(tq, tk, tv, p, n_units, s)
+                   : launch_pair_one<BF16, true, false, SPLIT, true>(tq, tk, tv, p, n_units, s);
+    if (causal)
+        return neg ? launch_pair_one<BF16, true, true, SPLIT, false>(tq, tk, tv, p, n_units, s)
+                   : launch_pair_one<BF16, true, false, SPLIT, false>(tq, tk, tv, p, n_units, s);
+    return neg ? launch_pair_one<BF16, false, true, SPLIT, false>(tq, tk, tv, p, n_units, s)
+               : launch_pair_one<BF16, false, false, SPLIT, false>(tq, tk, tv, p, n_units, s);
+}
+
 // Wide kernel ring depth: 64-key K/V stages beside the 128-row Q tile (~192 KB).
 template <int D>
 constexpr int kWideStages = (D == 256) ? 2 : 3;
@@ -360,13 +442,25 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int BH = B * Hkv;
     const int rows = (H / Hkv) * Sq;
     const bool bf16 = dtype == ATTN_BF16;
-    const bool wide = is_wide(D);
-    const int kv_keys = kv_tile_keys(D);
+    // D = 256 with more than one query tile of packed rows runs on CTA pairs (the
+    // D <= 128 geometry: 256-row units, 128-key tiles, each CTA holding half of every
+    // K tile); otherwise D = 192 / 256 run in the wide kernel.
+    const bool pair_path = D == 256 && rows > attn::BM;
+    const bool wide = is_wide(D) && !pair_path;
+    const int kv_keys = wide ? attn::wide::WBN : attn::BN;
+    const int q_units = wide ? attn::wide::WBM : attn::ROWS_PER_CTA;
     CUtensorMap tq, tk, tv;
-    if (!encode_qkv_map(&tq, q, D, rows, BH, bf16, attn::BM) ||
-        !encode_qkv_map(&tk, k, D, Sk, BH, bf16, kv_keys) ||
-        !encode_qkv_map(&tv, v, D, Sk, BH, bf16, kv_keys))
+    if (pair_path) {
+        // one box per half tile: Q 128 rows, K 64 keys (all 4 chunks); V 128 keys, 2 chunks
+        if (!encode_chunked_map(&tq, q, D, rows, BH, bf16, attn::BM, D / attn::CHUNK_ELEMS) ||
+            !encode_chunked_map(&tk, k, D, Sk, BH, bf16, 64, D / attn::CHUNK_ELEMS) ||
+            !encode_chunked_map(&tv, v, D, Sk, BH, bf16, attn::BN, 2))
+            return ATTN_ERR_TENSORMAP;
+    } else if (!encode_qkv_map(&tq, q, D, rows, BH, bf16, attn::BM) ||
+               !encode_qkv_map(&tk, k, D, Sk, BH, bf16, wide ? 64 : attn::BN) ||
+               !encode_qkv_map(&tv, v, D, Sk, BH, bf16, wide ? 64 : attn::BN)) {
         return ATTN_ERR_TENSORMAP;
+    }
 
     attn::Params p;
     p.o = o;
@@ -374,7 +468,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     p.Sq = rows;
     p.Sk = Sk;
     p.BH = BH;
-    p.n_qp = (rows + unit_rows(D) - 1) / unit_rows(D);  // query units (wide: tiles)
+    p.n_qp = (rows + q_units - 1) / q_units;  // query units (wide: single tiles)
     p.sq_head = Sq;
     p.d_out = D;
     p.causal_off = mask == ATTN_MASK_CAUSAL_BOTTOM_RIGHT ? Sk - Sq : 0;
@@ -396,11 +490,19 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     if (n_units > INT_MAX) return ATTN_ERR_SHAPE;
     const int grid = n_units < num_sms ? static_cast<int>(n_units) : num_sms;
     const bool c = mask != ATTN_MASK_NONE;
-    if (n_splits == 0)
+    if (n_splits == 0) {
+        if (pair_path)
+            return bf16 ? launch_pair<true, false>(tq, tk, tv, p, n_units, c, stream)
+                        : launch_pair<false, false>(tq, tk, tv, p, n_units, c, stream);
         return wide ? launch_wide<false>(tq, tk, tv, p, grid, D, bf16, c, stream)
                     : launch_any<false>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
-    rc = wide ? launch_wide<true>(tq, tk, tv, p, grid, D, bf16, c, stream)
-              : launch_any<true>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
+    }
+    if (pair_path)
+        rc = bf16 ? launch_pair<true, true>(tq, tk, tv, p, n_units, c, stream)
+                  : launch_pair<false, true>(tq, tk, tv, p, n_units, c, stream);
+    else
+        rc = wide ? launch_wide<true>(tq, tk, tv, p, grid, D, bf16, c, stream)
+                  : launch_any<true>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
     if (rc != ATTN_OK) return rc;
     return launch_merge(p.ws_o, p.ws_lse, o, lse, n_splits, static_cast<int64_t>(B) * H * Sq, D,
                         bf16, stream);
