@@ -72,30 +72,27 @@ bool encode_qkv_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool
     return r == CUDA_SUCCESS;
 }
 
-// The same tensor seen as 4-D (64 columns, S rows, D/64 column chunks, BH heads): a box
-// of 64 columns x box_rows rows x box_chunks chunks lands in shared memory chunk-major,
-// each chunk box_rows x 128 bytes in the 128-byte swizzle, as box_chunks 3-D boxes
-// would.  D a multiple of 64.
+// The same tensor seen as 4-D (cw columns, S rows, D/cw column chunks, BH heads): a box
+// of cw columns x box_rows rows x box_chunks chunks lands in shared memory chunk-major,
+// each chunk box_rows x (2 cw) bytes in the swizzle of that row size (cw = 64: 128-byte
+// swizzle; cw = 32: 64-byte swizzle), as box_chunks 3-D boxes would.  D a multiple of cw.
 bool encode_chunked_map(CUtensorMap* m, const void* base, int D, int S, int BH, bool bf16,
-                        int box_rows, int box_chunks) {
+                        int box_rows, int box_chunks, int cw) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(attn::CHUNK_ELEMS),
-                                static_cast<cuuint64_t>(S),
-                                static_cast<cuuint64_t>(D / attn::CHUNK_ELEMS),
-                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(cw), static_cast<cuuint64_t>(S),
+                                static_cast<cuuint64_t>(D / cw), static_cast<cuuint64_t>(BH)};
     const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
-                                   static_cast<cuuint64_t>(attn::CHUNK_ELEMS) * 2,
+                                   static_cast<cuuint64_t>(cw) * 2,
                                    static_cast<cuuint64_t>(S) * D * 2};
-    const cuuint32_t box[4] = {static_cast<cuuint32_t>(attn::CHUNK_ELEMS),
-                               static_cast<cuuint32_t>(box_rows),
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(cw), static_cast<cuuint32_t>(box_rows),
                                static_cast<cuuint32_t>(box_chunks), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUresult r =
         fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+           cw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -290,14 +287,15 @@ int launch_wide_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-// D = 256 on CTA pairs: clusters of two CTAs, the grid sized to the clusters that can
-// be resident at once (a persistent grid; the pair walks its units).
-template <bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
+// D = 192 / 256 on CTA pairs: clusters of two CTAs, the grid sized to the clusters that
+// can be resident at once (a persistent grid; the pair walks its units).
+template <int PD, bool BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
 int launch_pair_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const attn::Params& p, int64_t n_units, cudaStream_t stream) {
-    constexpr int NSK = 3, NSV = 2;  // K / V ring stages (224 KB with Q)
-    auto kern = attn::pair::attn_fwd_pair_kernel<NSK, NSV, BF16, CAUSAL, NEG, SPLIT, GEN>;
-    constexpr int smem = attn::pair::Layout<NSK, NSV>::ALLOC;
+    // K / V ring stages: D = 256 3 + 2 (224 KB with Q), D = 192 3 + 3 (192 KB)
+    constexpr int NSK = 3, NSV = PD == 256 ? 2 : 3;
+    auto kern = attn::pair::attn_fwd_pair_kernel<PD, NSK, NSV, BF16, CAUSAL, NEG, SPLIT, GEN>;
+    constexpr int smem = attn::pair::Layout<PD, NSK, NSV>::ALLOC;
     static int max_clusters[kMaxDevices];  // 0: not yet known
     static std::mutex mu;
     int dev = 0;
@@ -331,18 +329,28 @@ int launch_pair_one(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensor
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH;
 }
 
-template <bool BF16, bool SPLIT>
-int launch_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const attn::Params& p, int64_t n_units, bool causal, cudaStream_t s) {
+template <int PD, bool BF16, bool SPLIT>
+int launch_pair_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                  const attn::Params& p, int64_t n_units, bool causal, cudaStream_t s) {
     const bool neg = p.scale_log2 < 0.f;
     if (causal && (p.causal_off != 0 || p.sq_head != p.Sq))
-        return neg ? launch_pair_one<BF16, true, true, SPLIT, true>(tq, tk, tv, p, n_units, s)
-                   : launch_pair_one<BF16, true, false, SPLIT, true>(tq, tk, tv, p, n_units, s);
+        return neg ? launch_pair_one<PD, BF16, true, true, SPLIT, true>(tq, tk, tv, p, n_units, s)
+                   : launch_pair_one<PD, BF16, true, false, SPLIT, true>(tq, tk, tv, p, n_units, s);
     if (causal)
-        return neg ? launch_pair_one<BF16, true, true, SPLIT, false>(tq, tk, tv, p, n_units, s)
-                   : launch_pair_one<BF16, true, false, SPLIT, false>(tq, tk, tv, p, n_units, s);
-    return neg ? launch_pair_one<BF16, false, true, SPLIT, false>(tq, tk, tv, p, n_units, s)
-               : launch_pair_one<BF16, false, false, SPLIT, false>(tq, tk, tv, p, n_units, s);
+        return neg ? launch_pair_one<PD, BF16, true, true, SPLIT, false>(tq, tk, tv, p, n_units, s)
+                   : launch_pair_one<PD, BF16, true, false, SPLIT, false>(tq, tk, tv, p, n_units, s);
+    return neg ? launch_pair_one<PD, BF16, false, true, SPLIT, false>(tq, tk, tv, p, n_units, s)
+               : launch_pair_one<PD, BF16, false, false, SPLIT, false>(tq, tk, tv, p, n_units, s);
+}
+
+template <bool SPLIT>
+int launch_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const attn::Params& p, int64_t n_units, int D, bool bf16, bool causal,
+                cudaStream_t s) {
+    if (D == 192) return bf16 ? launch_pair_d<192, true, SPLIT>(tq, tk, tv, p, n_units, causal, s)
+                              : launch_pair_d<192, false, SPLIT>(tq, tk, tv, p, n_units, causal, s);
+    return bf16 ? launch_pair_d<256, true, SPLIT>(tq, tk, tv, p, n_units, causal, s)
+                : launch_pair_d<256, false, SPLIT>(tq, tk, tv, p, n_units, causal, s);
 }
 
 // Wide kernel ring depth: 64-key K/V stages beside the 128-row Q tile (~192 KB).
@@ -442,19 +450,22 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int BH = B * Hkv;
     const int rows = (H / Hkv) * Sq;
     const bool bf16 = dtype == ATTN_BF16;
-    // D = 256 with more than one query tile of packed rows runs on CTA pairs (the
+    // D = 192 / 256 with more than one query tile of packed rows run on CTA pairs (the
     // D <= 128 geometry: 256-row units, 128-key tiles, each CTA holding half of every
-    // K tile); otherwise D = 192 / 256 run in the wide kernel.
-    const bool pair_path = D == 256 && rows > attn::BM;
+    // K and V tile); with fewer rows (decoding) they run in the wide kernel.
+    const bool pair_path = is_wide(D) && rows > attn::BM;
     const bool wide = is_wide(D) && !pair_path;
     const int kv_keys = wide ? attn::wide::WBN : attn::BN;
     const int q_units = wide ? attn::wide::WBM : attn::ROWS_PER_CTA;
     CUtensorMap tq, tk, tv;
     if (pair_path) {
-        // one box per half tile: Q 128 rows, K 64 keys (all 4 chunks); V 128 keys, 2 chunks
-        if (!encode_chunked_map(&tq, q, D, rows, BH, bf16, attn::BM, D / attn::CHUNK_ELEMS) ||
-            !encode_chunked_map(&tk, k, D, Sk, BH, bf16, 64, D / attn::CHUNK_ELEMS) ||
-            !encode_chunked_map(&tv, v, D, Sk, BH, bf16, attn::BN, 2))
+        // one box per half tile: Q 128 rows and K 64 keys, all 64-column chunks; V 128
+        // keys, this CTA's D/2 columns (64-column chunks at D = 256, 32-column at 192)
+        const int vcw = D == 256 ? 64 : 32;
+        const int nch = D / attn::CHUNK_ELEMS;
+        if (!encode_chunked_map(&tq, q, D, rows, BH, bf16, attn::BM, nch, attn::CHUNK_ELEMS) ||
+            !encode_chunked_map(&tk, k, D, Sk, BH, bf16, 64, nch, attn::CHUNK_ELEMS) ||
+            !encode_chunked_map(&tv, v, D, Sk, BH, bf16, attn::BN, D / 2 / vcw, vcw))
             return ATTN_ERR_TENSORMAP;
     } else if (!encode_qkv_map(&tq, q, D, rows, BH, bf16, attn::BM) ||
                !encode_qkv_map(&tk, k, D, Sk, BH, bf16, wide ? 64 : attn::BN) ||
@@ -491,15 +502,12 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int grid = n_units < num_sms ? static_cast<int>(n_units) : num_sms;
     const bool c = mask != ATTN_MASK_NONE;
     if (n_splits == 0) {
-        if (pair_path)
-            return bf16 ? launch_pair<true, false>(tq, tk, tv, p, n_units, c, stream)
-                        : launch_pair<false, false>(tq, tk, tv, p, n_units, c, stream);
+        if (pair_path) return launch_pair<false>(tq, tk, tv, p, n_units, D, bf16, c, stream);
         return wide ? launch_wide<false>(tq, tk, tv, p, grid, D, bf16, c, stream)
                     : launch_any<false>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);
     }
     if (pair_path)
-        rc = bf16 ? launch_pair<true, true>(tq, tk, tv, p, n_units, c, stream)
-                  : launch_pair<false, true>(tq, tk, tv, p, n_units, c, stream);
+        rc = launch_pair<true>(tq, tk, tv, p, n_units, D, bf16, c, stream);
     else
         rc = wide ? launch_wide<true>(tq, tk, tv, p, grid, D, bf16, c, stream)
                   : launch_any<true>(tq, tk, tv, p, grid, kernel_d(D), bf16, c, stream);

@@ -1,20 +1,23 @@
-// attn_fwd_pair_kernel.cuh -- the fused attention forward pass for head dimension 256 on
-// a pair of CTAs (a cluster of two, one per SM) whose tensor cores run each MMA
-// together (tcgen05 cta_group::2, M = 256).
+// attn_fwd_pair_kernel.cuh -- the fused attention forward pass for head dimensions 192
+// and 256 on a pair of CTAs (a cluster of two, one per SM) whose tensor cores run each
+// MMA together (tcgen05 cta_group::2, M = 256).
 //
-// Why: at D = 256 one CTA can hold only one 128-row query tile (its O takes 256 of the
+// Why: at these D one CTA can hold only one 128-row query tile (its O takes D of the
 // 512 TMEM columns), so every K/V byte it loads feeds 128 query rows, and the 64-key
 // tiles that fit beside its Q make the S products N = 64 MMAs, which run into the
 // per-instruction issue floor.  A pair runs a 256-row query block as one M = 256
 // problem: CTA r holds query rows 128r .. 128r + 127 of the block, and of every
 // 128-key tile it loads only its half of the B operands -- keys 64r .. 64r + 63 of K
-// (S = Q K^T, N = 128 split over the pair) and columns 128r .. 128r + 127 of V
-// (O = P V, N = D = 256 split over the pair).  Per SM that halves the K/V bytes per
-// FLOP, and S runs as N = 128 MMAs.
+// (S = Q K^T, N = 128 split over the pair) and columns (D/2)r .. (D/2)r + D/2 - 1 of V
+// (O = P V, N = D split over the pair).  Per SM that halves the K/V bytes per FLOP,
+// and S runs as N = 128 MMAs.  V's halves are 128 columns at D = 256 (two chunks of 64
+// in the 128-byte swizzle) and 96 at D = 192 (three chunks of 32 in the 64-byte
+// swizzle: a half of 96 columns does not split into 64-column chunks).
 //
-// Each CTA: Q (64 KB), a ring of NSK K halves (32 KB each) and one of NSV V halves
-// (32 KB each) in shared memory (3 + 2 stages: 224 KB; K gets the extra stage, its
-// load has one tile less of lead than V's in the MMA order below); two 128-column S buffers (0, 128) and O (256 .. 511) in tensor memory.
+// Each CTA: Q (D/64 chunks of 16 KB), a ring of NSK K halves and one of NSV V halves in
+// shared memory (D = 256: 3 + 2 stages of 32 KB, 224 KB with Q -- K gets the extra
+// stage; D = 192: 3 + 3 stages of 24 KB); two 128-column S buffers (0, 128) and O (from
+// column 256) in tensor memory.
 // Rank 0 issues every MMA (S_0 S_1 | PV_0 S_2 | PV_1 S_3 | ..., KV tile j in S buffer
 // j % 2); both CTAs run a TMA producer, four softmax warps (thread = row, 128 scores a
 // tile) and four epilogue warps on their own rows.  Hand-offs across the pair:
@@ -38,19 +41,28 @@
 namespace attn {
 namespace pair {
 
-constexpr int PD = 256;                  // head dimension
 constexpr int NUM_THREADS = 384;
 constexpr int Q_CHUNK = 128 * 128;       // 128 query rows x 128 bytes
 constexpr int K_CHUNK = 64 * 128;        // 64 keys x 128 bytes (this CTA's half of a tile)
-constexpr int V_CHUNK = 128 * 128;       // 128 keys x 64 columns
 constexpr uint32_t TMEM_O = 256;         // O columns; S buffers at 0 and 128
 
-template <int NSK, int NSV>
+// V halves: chunks of V_CW columns (128 keys each), MN-major in the matching swizzle.
+template <int PD>
+struct VGeo {
+    static_assert(PD == 192 || PD == 256, "head dim 192 or 256");
+    static constexpr int V_CW = PD == 256 ? 64 : 32;       // columns per chunk
+    static constexpr int VCH = PD / 2 / V_CW;              // chunks per CTA (2 or 3)
+    static constexpr int V_CHUNK = 128 * V_CW * 2;         // 16 KB or 8 KB
+    static constexpr uint32_t SBO = 8 * V_CW * 2;          // bytes per 8-key group
+    static constexpr uint32_t KSTEP = (16 * V_CW * 2) >> 4;  // 16 keys, descriptor units
+};
+
+template <int PD, int NSK, int NSV>
 struct Layout {
-    static constexpr int NCH = PD / CHUNK_ELEMS;        // 4 chunks of 64 columns
-    static constexpr int Q_BYTES = NCH * Q_CHUNK;       // 64 KB
-    static constexpr int K_BYTES = NCH * K_CHUNK;       // 32 KB
-    static constexpr int V_BYTES = 2 * V_CHUNK;         // 32 KB (this CTA's 128 columns)
+    static constexpr int NCH = PD / CHUNK_ELEMS;        // 64-column chunks of Q and K
+    static constexpr int Q_BYTES = NCH * Q_CHUNK;
+    static constexpr int K_BYTES = NCH * K_CHUNK;
+    static constexpr int V_BYTES = VGeo<PD>::VCH * VGeo<PD>::V_CHUNK;  // D/2 columns
     static constexpr int Q_OFF = 0;
     static constexpr int K_OFF = Q_OFF + Q_BYTES;
     static constexpr int V_OFF = K_OFF + NSK * K_BYTES;
@@ -95,12 +107,13 @@ __device__ __forceinline__ int pair_unit_of(int r, int n_units) {
     return u < n_units ? u : -1;
 }
 
-template <int NSK, int NSV, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
+template <int PD, int NSK, int NSV, bool IS_BF16, bool CAUSAL, bool NEG, bool SPLIT, bool GEN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
-    using L = Layout<NSK, NSV>;
+    using L = Layout<PD, NSK, NSV>;
+    using VG = VGeo<PD>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = ptx::smem_u32(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -314,9 +327,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             constexpr uint32_t idesc_qk = ptx::idesc_f16(fmt, 2 * BM, BN, 0);
             constexpr uint32_t idesc_pv = ptx::idesc_f16(fmt, 2 * BM, PD, 1);
             constexpr uint32_t desc_hi = ptx::smem_desc_hi_sw128(1024);
+            constexpr uint32_t v_hi = PD == 256 ? ptx::smem_desc_hi_sw128(VG::SBO)
+                                                : ptx::smem_desc_hi_sw64(VG::SBO);
             const uint32_t dq = ptx::smem_desc_lo(sQ, 16);
             const uint32_t dk0 = ptx::smem_desc_lo(sK, 16);
-            const uint32_t dv0 = ptx::smem_desc_lo(sV, V_CHUNK);
+            const uint32_t dv0 = ptx::smem_desc_lo(sV, VG::V_CHUNK);
             // completion to this CTA's barrier and to the same barrier of rank 1
             auto commit2 = [&](uint32_t bar) {
                 ptx::mma_commit_pair(bar);
@@ -337,20 +352,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 commit2(B_SF(b));
             };
-            // O (+)= P_b V (M = 256, N = 256): K steps of 16 keys, 8 TMEM columns of P
-            // and 2 KB of each V chunk
+            // O (+)= P_b V (M = 256, N = D): K steps of 16 keys, 8 TMEM columns of P and
+            // 16 rows of each V chunk
             auto issue_pv = [&](int b, int slot, bool first) {
+                constexpr uint32_t K1 = VG::KSTEP;
                 const uint32_t vd = dv0 + static_cast<uint32_t>(slot) * (L::V_BYTES >> 4);
                 const uint32_t a_tmem = tmem + 128u * b;
                 const uint32_t d_tmem = tmem + TMEM_O;
-                ptx::mma2_ts_off<0, 0>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, first ? 0u : 1u);
-                ptx::mma2_ts_off<8, 128>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
-                ptx::mma2_ts_off<16, 256>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
-                ptx::mma2_ts_off<24, 384>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
-                ptx::mma2_ts_off<32, 512>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
-                ptx::mma2_ts_off<40, 640>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
-                ptx::mma2_ts_off<48, 768>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
-                ptx::mma2_ts_off<56, 896>(d_tmem, a_tmem, vd, desc_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<0, 0>(d_tmem, a_tmem, vd, v_hi, idesc_pv, first ? 0u : 1u);
+                ptx::mma2_ts_off<8, K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<16, 2 * K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<24, 3 * K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<32, 4 * K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<40, 5 * K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<48, 6 * K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
+                ptx::mma2_ts_off<56, 7 * K1>(d_tmem, a_tmem, vd, v_hi, idesc_pv, 1u);
             };
             bool ok = true;
             uint32_t kv = 0, nu = 0, ut = 0;
@@ -406,9 +422,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         // ================================================================ producers
         // Both CTAs load their halves (K_0 .. K_{NSK-1}, then V_j, K_{j+NSK}), the bytes
         // counted on rank 0's full barriers; rank 0 posts the expected bytes of both
-        // halves.  The tensor maps see each operand as (64 columns, rows, column chunk,
-        // head), so one box lands a whole half tile chunk-major: Q 128 rows x 4 chunks,
-        // K 64 keys x 4 chunks, V 128 keys x this CTA's 2 chunks.
+        // halves.  The tensor maps see each operand as (chunk columns, rows, column
+        // chunk, head), so one box lands a whole half tile chunk-major: Q 128 rows and K
+        // 64 keys x D/64 chunks of 64 columns, V 128 keys x this CTA's chunks.
         if (lane == 0) {
             const bool load_q = !(p.flags & FLAG_SKIP_Q_LOAD);
             const int rk = static_cast<int>(rank);
@@ -429,7 +445,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (!wait_cl(ctx, B_VE(s), ((pos / NSV) & 1) ^ 1)) return false;
                 if (lead) ptx::mbar_arrive_expect_tx(B_VF(s), 2 * L::V_BYTES);
                 ptx::tma_load_4d_pair(sV + s * L::V_BYTES, &tm_v, ptx::mapa_shared(B_VF(s), 0), 0,
-                                      kt * BN, 2 * rk, bh);
+                                      kt * BN, VG::VCH * rk, bh);
                 last_v = pos;
                 return true;
             };

@@ -213,6 +213,12 @@ __host__ __device__ constexpr uint32_t smem_desc_hi_sw128(uint32_t sbo_bytes) {
     return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
 
+// High word for the 64-byte swizzle (layout 4): used for MN-major tiles of 32-element
+// chunks (8-row groups of 512 bytes).
+__host__ __device__ constexpr uint32_t smem_desc_hi_sw64(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (4u << 29);
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 // fmt: 0 = f16, 1 = bf16; b_mn_major: B operand stored MN-major.
 __host__ __device__ constexpr uint32_t idesc_f16(uint32_t fmt, uint32_t M, uint32_t N,

@@ -79,7 +79,8 @@ enum {
  *   lse    device, [B,H,Sq] fp32, written; may be NULL (not written)
  *   B, H, Sq, Sk >= 1; B*H, Sq, Sk <= 2^24; D in {64, 80, 96, 112, 128, 192, 256}
  *          (80, 96 and 112 run as 128 with the missing columns read as zeros: exact, at
- *          the cost of the padded work; 192 and 256 run in a kernel of their own with
+ *          the cost of the padded work; 192 and 256 run on pairs of CTAs that share
+ *          each MMA, or, for at most 128 query rows per K/V head, in a kernel with
  *          128-row query tiles and 64-key K/V tiles)
  *   causal 0: every key visible; nonzero: key j visible to query i iff j <= i
  *   scale  finite multiplier of q.k (e.g. 1/sqrt(D)); |scale*q.k| must fit fp32
