@@ -50,3 +50,30 @@ def test_debug_entry_without_flags_is_the_normal_pass():
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert af.attn_fwd_status() == 0
+
+
+@pytest.mark.parametrize("D,Sq", [(256, 300), (192, 300), (256, 64)])
+def test_starved_pipeline_on_the_wide_head_dimensions(D, Sq):
+    """The same starved pipeline on the CTA-pair kernel (D = 192 / 256 with more than 128
+    rows: both CTAs of every pair skip their Q loads; rank 0's MMA thread gives up on Q,
+    rank 1's softmax gives up on S, each CTA's other roles see its flag, and the two
+    meet at the cluster barrier and leave) and on the wide kernel (a decode shape)."""
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, Sq, 500, D, "bf16", 24))
+    o = torch.zeros_like(q)
+    lse = torch.zeros((1, 2, Sq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert af.attn_fwd_status() == 0
+    t0 = time.monotonic()
+    rc = af.attn_fwd_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           lse.data_ptr(), 1, 2, Sq, 500, D, 1, 0.07, af.ATTN_BF16, stream, 1)
+    assert rc == af.ATTN_OK
+    status = af.attn_fwd_status()
+    elapsed = time.monotonic() - t0
+    assert status == af.ATTN_ERR_TIMEOUT
+    assert 1.0 < elapsed < 30.0
+    assert af.attn_fwd_status() == 0
+    check_full(1, 2, 300, 400, 64, "f16", False, seed=25)
+    # and the kernel itself runs normally again
+    o2, l2 = af.attention(q, k, v, causal=True, scale=0.07)
+    torch.cuda.synchronize()
+    assert af.attn_fwd_status() == 0 and torch.isfinite(o2.float()).all()
