@@ -154,7 +154,8 @@ bool head_dim_ok(int D) {
 }
 int kernel_d(int D) { return D <= 64 ? 64 : D <= 128 ? 128 : D; }
 bool is_wide(int D) { return D > 128; }
-// query rows and keys per work unit and KV tile of the kernel that runs D
+// query rows per work unit, at the least over the kernels that can run D (the bound
+// on the unit count checked by validate)
 int unit_rows(int D) { return is_wide(D) ? attn::wide::WBM : attn::ROWS_PER_CTA; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {

@@ -1,7 +1,9 @@
 // attn_fwd_wide_kernel.cuh -- the fused attention forward pass for head dimensions 192
-// and 256, where two 128-row query tiles per CTA no longer fit: their O accumulators
-// (2 x D fp32 columns) plus S exceed the 512 tensor-memory columns, and a 64 KB query
-// tile leaves shared memory for only one 128-key K/V stage.
+// and 256 on a single CTA, where two 128-row query tiles per CTA no longer fit: their O
+// accumulators (2 x D fp32 columns) plus S exceed the 512 tensor-memory columns, and a
+// 64 KB query tile leaves shared memory for only one 128-key K/V stage.  The library runs
+// it for at most 128 packed query rows per K/V head (decoding); larger problems run on
+// CTA pairs (attn_fwd_pair_kernel.cuh), which share every K/V tile between 256 rows.
 //
 // Tile plan: one 128-row query tile per CTA and KV tiles of 64 keys, so the ring holds
 // 2 (D = 256) or 3 (D = 192) K/V stages.  Tensor memory: two 64-column S buffers
