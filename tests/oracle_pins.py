@@ -291,8 +291,37 @@ def pin_grouped_heads_torch(lib):
         assert np.array_equal(ro, o[idx]) and np.array_equal(rl, lse[idx])
 
 
+def pin_product_head_dims(lib):
+    """PyTorch's float64 math SDPA at every head dimension the CUDA path accepts (64, 80,
+    96, 112, 128, 192, 256), all three masks, Sq < Sk and Sq > Sk."""
+    for n, D in enumerate((64, 80, 96, 112, 128, 192, 256)):
+        for (Sq, Sk) in ((5, 9), (9, 4)):
+            q = _rand((1, 2, Sq, D), 80 + n)
+            k = _rand((1, 2, Sk, D), 90 + n)
+            v = _rand((1, 2, Sk, D), 100 + n)
+            scale = 1.0 / math.sqrt(D)
+            tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+            masks = ((oracle.NO_MASK, torch.ones(Sq, Sk, dtype=torch.bool)),
+                     (oracle.CAUSAL_TOP_LEFT, torch.ones(Sq, Sk, dtype=torch.bool).tril()),
+                     (oracle.CAUSAL_BOTTOM_RIGHT,
+                      torch.tril(torch.ones(Sq, Sk, dtype=torch.bool), diagonal=Sk - Sq)))
+            for mask, allowed in masks:
+                o, lse = oracle.attn_ref_ex(q, k, v, mask, scale, lib=lib)
+                s = scale * torch.einsum("bhid,bhjd->bhij", tq, tk)
+                s = s.masked_fill(~allowed, float("-inf"))
+                np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(),
+                                           rtol=0, atol=1e-12)
+                seen = allowed.any(dim=1)   # rows with at least one visible key
+                with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+                    ref = torch.nn.functional.scaled_dot_product_attention(
+                        tq[:, :, seen], tk, tv, attn_mask=allowed[seen], scale=scale)
+                np.testing.assert_allclose(o[:, :, seen.numpy()], ref.numpy(), rtol=0, atol=1e-12)
+                assert (o[:, :, ~seen.numpy()] == 0.0).all()
+
+
 ALL_PINS = [pin_single_key, pin_zero_query, pin_constant_value, pin_causal_first_row,
             pin_hand_2x2, pin_hand_3x2_causal, pin_one_hot_huge_margin,
             pin_probability_rows, pin_permutation, pin_key_shift, pin_linear_in_value,
             pin_torch_sdpa, pin_rows_match_whole,
-            pin_bottom_right_closed_forms, pin_bottom_right_torch, pin_grouped_heads_torch]
+            pin_bottom_right_closed_forms, pin_bottom_right_torch, pin_grouped_heads_torch,
+            pin_product_head_dims]
