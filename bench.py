@@ -63,8 +63,9 @@ def parse():
     ap.add_argument("--profile-once", action="store_true",
                     help="launch each pass of the workload once and exit (for ncu captures)")
     ap.add_argument("--profile-extra", default=None,
-                    help="with --profile-once: a DEC*, SMX* or GEMM* workload instead, optionally "
-                         "scaled down as NAME:rows (M for GEMM*, rows for SMX*, B for DEC*)")
+                    help="with --profile-once: a DEC*, SMX*, GEMM* or WD* workload instead, "
+                         "optionally scaled down as NAME:n (M for GEMM*, rows for SMX*, B for "
+                         "DEC*, H for WD*)")
     return ap.parse_args()
 
 
