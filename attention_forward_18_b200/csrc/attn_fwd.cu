@@ -99,7 +99,7 @@ bool encode_chunked_map(CUtensorMap* m, const void* base, int D, int S, int BH, 
 // Per-device facts checked once: compute capability 10.x and the SM count (the
 // persistent grid has one CTA per SM).
 int check_device(int* num_sms) {
-    static int verdict[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
+    static int dev_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
     static int sms[kMaxDevices];
     static std::mutex mu;
     int dev = -1;
@@ -108,18 +108,18 @@ int check_device(int* num_sms) {
         return ATTN_ERR_DEVICE;
     }
     std::lock_guard<std::mutex> lock(mu);
-    if (verdict[dev] == 0) {
+    if (dev_ok[dev] == 0) {
         int major = 0, count = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_DEVICE;
         }
-        verdict[dev] = (major == 10 && count > 0) ? 1 : -1;
+        dev_ok[dev] = (major == 10 && count > 0) ? 1 : -1;
         sms[dev] = count;
     }
     if (num_sms) *num_sms = sms[dev];
-    return verdict[dev] == 1 ? ATTN_OK : ATTN_ERR_DEVICE;
+    return dev_ok[dev] == 1 ? ATTN_OK : ATTN_ERR_DEVICE;
 }
 
 // Device address of g_noalloc_scratch on the current device, looked up once per
