@@ -758,7 +758,7 @@ def main():
             line["extra"] = extra_workloads(["C3", "C4", "C5", "WD192", "WD256"], world)
             line["extra"]["cuda_graph"] = graph_launches(["C1", "C2"])
             line["extra"]["decode_splitkv"] = decode_workloads(
-                ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])
+                ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5", "DEC6"])
             line["extra"]["prefill_grouped_bottom_right"] = prefill_workloads(["PRE1"])
             line["extra"]["row_softmax"] = softmax_workloads(["SMX1", "SMX2", "SMX3"])
             line["extra"]["gemm_bias_act"] = gemm_workloads(["GEMM1", "GEMM2", "GEMM3"])

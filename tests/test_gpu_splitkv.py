@@ -117,7 +117,7 @@ def test_workspace_too_small_is_rejected_on_device():
     assert rc == af.ATTN_ERR_WORKSPACE
 
 
-@pytest.mark.parametrize("name", ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5"])
+@pytest.mark.parametrize("name", ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5", "DEC6"])
 def test_decode_workloads_in_bench_configuration(name):
     """The benchmark's decode workloads with the split count the benchmark uses (DEC5
     with grouped K/V heads through attn_fwd_ex): every row against the oracle (sampled

@@ -85,6 +85,8 @@ DECODE_WORKLOADS = {
                      note="batch of 16, D=64, 4K keys"),
     "DEC5": Workload("DEC5", 8, 32, 1, 8192, 128, "bf16", (False,), 9, Hkv=8,
                      note="grouped heads: 32 query heads on 8 K/V heads, batch 8, 8K keys"),
+    "DEC6": Workload("DEC6", 4, 16, 1, 16384, 256, "bf16", (False,), 32,
+                     note="head dimension 256, batch of 4, one query row per head, 16K keys"),
 }
 
 
