@@ -3,6 +3,9 @@ seeded inputs and compare with the fp64 oracle element by element.
 
 Tolerances (stated for the fused forward with 16-bit inputs and fp32
 accumulation): max |O_gpu - O_ref| <= 2e-2 and max |LSE_gpu - LSE_ref| <= 1e-3."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -42,10 +45,21 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return rep
 
 
+def record(what, rep):
+    """Append a comparison report to the JSON-lines file named by ATTN_PARITY_REPORT
+    (when set), so a run can keep the measured errors of its full-size checks."""
+    path = os.environ.get("ATTN_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": what, **rep}) + "\n")
+
+
 def check_full(B, H, Sq, Sk, D, dtype, causal, seed, k_scale=1.0, scale=None):
     scale = (1.0 / np.sqrt(D)) if scale is None else scale
     q, k, v = make_qkv(B, H, Sq, Sk, D, dtype, seed, k_scale)
     o, lse = run_gpu(q, k, v, causal, scale)
     o_ref, lse_ref = oracle.attn_ref(q.double().numpy(), k.double().numpy(),
                                      v.double().numpy(), causal, scale)
-    return compare(o, lse, o_ref, lse_ref, f"B{B} H{H} Sq{Sq} Sk{Sk} D{D} {dtype} c{causal}")
+    what = f"B{B} H{H} Sq{Sq} Sk{Sk} D{D} {dtype} c{causal}"
+    rep = compare(o, lse, o_ref, lse_ref, what)
+    return rep

@@ -6,8 +6,8 @@ import torch
 
 import attention_forward_18_b200 as af
 import oracle
-from parity import O_TOL, LSE_TOL, check_full, compare, run_gpu
-from workloads import WORKLOADS, make_inputs, make_qkv, sample_rows
+from parity import O_TOL, LSE_TOL, check_full, compare, record, run_gpu
+from workloads import WORKLOADS, make_inputs, make_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -15,13 +15,6 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("causal", [False, True])
 def test_tiny_workload_whole(causal):
     w = WORKLOADS["C1"]
-    check_full(w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, causal, w.seed)
-
-
-@pytest.mark.parametrize("causal", [False, True])
-def test_bench_workload_whole(causal):
-    """The benchmark's workload (B=4, H=16, S=1024, D=64, fp16), every element."""
-    w = WORKLOADS["C2"]
     check_full(w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, causal, w.seed)
 
 
@@ -37,24 +30,45 @@ def test_ragged_shapes(Sq, Sk, causal, dtype, D):
     check_full(2, 3, Sq, Sk, D, dtype, causal, seed=Sq * 7 + Sk)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_bench_workload_whole(causal):
+    """C2 (B=4, H=16, S=1024, D=64, fp16), every element, both passes."""
+    w = WORKLOADS["C2"]
+    rep = check_full(w.B, w.H, w.Sq, w.Sk, w.D, w.dtype, causal, w.seed)
+    record(f"C2 causal={causal}", rep)
+
+
 @pytest.mark.parametrize("name", ["C3", "C4", "C5"])
-def test_large_workloads_sampled_rows(name):
-    """Full-size workloads in the benchmark's launch configuration; sampled rows
-    (edges, every tile boundary of one head, random rows) against the oracle row by
-    row, and at every position the properties that hold at any size."""
+def test_large_workloads_every_element(name):
+    """The full-size workloads of the benchmark step, launched as the benchmark launches
+    them, every element of O and LSE against the oracle: its row entry point (each
+    row's scores materialised in fp64, masked, softmaxed, times V) over every (b, h, i),
+    a few heads per call to bound host memory."""
     w = WORKLOADS[name]
     q, k, v = make_inputs(w)
+    qd, kd, vd = q.double().numpy(), k.double().numpy(), v.double().numpy()
     for causal in w.causal:
         o, lse = run_gpu(q, k, v, causal, w.scale)
-        assert np.isfinite(o).all() and np.isfinite(lse).all()
-        # O is a convex combination of V rows: |O| <= max |V| per head and feature
-        vmax = v.abs().amax(dim=2).double().numpy()            # [B,H,D]
-        assert (np.abs(o) <= vmax[:, :, None, :] + O_TOL).all()
-        rows = sample_rows(w.B, w.H, w.Sq, 96, seed=w.seed)
-        ro, rl = oracle.attn_ref_rows(q.double().numpy(), k.double().numpy(),
-                                      v.double().numpy(), rows, causal, w.scale)
-        idx = tuple(np.array(rows).T)
-        compare(o[idx], lse[idx], ro, rl, f"{name} causal={causal}")
+        o = o.reshape(w.B * w.H, w.Sq, w.D)
+        lse = lse.reshape(w.B * w.H, w.Sq)
+        per_call = max(1, (1 << 16) // w.Sq)       # heads per oracle call
+        total = {"max_dO": 0.0, "max_dLSE": 0.0, "rows": 0}
+        for h0 in range(0, w.B * w.H, per_call):
+            hs = np.arange(h0, min(h0 + per_call, w.B * w.H))
+            bh = np.repeat(hs, w.Sq)
+            rows = np.stack([bh // w.H, bh % w.H, np.tile(np.arange(w.Sq), len(hs))], axis=1)
+            ro, rl = oracle.attn_ref_rows(qd, kd, vd, rows, causal, w.scale)
+            rep = compare(o[hs].reshape(-1, w.D), lse[hs].reshape(-1), ro, rl,
+                          f"{name} causal={causal} heads {h0}..{hs[-1]}")
+            total["rows"] += len(rows)
+            if rep["max_dO"] >= total["max_dO"]:
+                r = rows[rep["worst"][0]]
+                total.update(max_dO=rep["max_dO"], worst_bhid=[int(r[0]), int(r[1]), int(r[2]),
+                                                               int(rep["worst"][1])],
+                             abs_O_at_worst=rep["|O| at worst"])
+            total["max_dLSE"] = max(total["max_dLSE"], rep["max_dLSE"])
+        assert total["rows"] == w.B * w.H * w.Sq
+        record(f"{name} causal={causal} (every element)", total)
 
 
 def test_lse_pointer_may_be_null():
