@@ -1,29 +1,38 @@
 """Benchmark of the fused attention forward pass on B200: prints ONE JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
-                    [--workload C2] [--no-extra]
+                    [--workload step|C1|C2|C3|C4|C5] [--no-extra]
 
-A step is one pass of the whole path over the workload: for the default workload
-(B=4, H=16, Sq=Sk=1024, D=64, fp16, seed 1) a non-causal pass and a causal pass on
-the same tensors, each one launch of the CUDA kernel through the C ABI.  The metric
-is TFLOP/s with FLOPs = 4*B*H*Sq*Sk*D per pass, halved for causal.
+A step is one pass over each of the three large workloads, each pass one launch of
+the CUDA kernel through the C ABI, all bf16 with head dimension 128:
+
+    C3  B=2 H=32 Sq=Sk=4096   causal                       seed 2
+    C4  B=8 H=32 Sq=Sk=2048   non-causal, K scaled by 3    seed 3
+    C5  B=1 H=16 Sq=Sk=16384  causal (long context)        seed 4
+
+The metric is TFLOP/s with FLOPs = 4*B*H*Sq*Sk*D per pass, halved for causal; `value`
+is the step's FLOPs over the step's time.  `--workload C2` (or another single
+workload) times that workload's passes instead.
 
 Timing: inputs resident in device memory; W untimed warm-up steps; then exactly K
-steps, each bracketed by CUDA events on the launching stream, with a 256 MB buffer
-written between steps so every step starts with a cold L2 (the workload's 25 MB of
-inputs would otherwise stay in the 126 MB L2); barrier + synchronize on both sides;
-the max over ranks of the summed step time.  Multi-GPU runs (torchrun, one rank per
-GPU) give every rank its own copy of the workload (weak scaling, no collective on
-the data path).
+steps with CUDA events around every pass on the launching stream; barrier +
+synchronize on both sides; the max over ranks of the summed step time.  Every pass of
+the default step reads at least 201 MB of Q/K/V, more than the 126 MB L2, so no pass
+finds its inputs in L2 (no flush is needed); a workload whose inputs fit in L2 gets a
+256 MB read between steps.  Multi-GPU runs (torchrun, one rank per GPU) give every
+rank its own copy of the workload (weak scaling, no collective on the data path).
 
-Also reported: `e2e` (the same steps through attn_fwd_host from pinned host buffers,
+Also reported: `e2e` (the same step through attn_fwd_host from pinned host buffers,
 copies included), `roofline` (the dominant kernel's achieved TFLOP/s against the
-measured dense bf16 peak), `cpu_baseline` (the fp64 CPU oracle on a bounded sample
-of the workload, rank 0 at N=1), `clocks` (NVML samples taken during the timed
-region) and `extra` (the other large workloads, and the split-KV pass on
-decode-shaped workloads, timed the same way, outside the timed region).
+measured dense bf16 peak, with its DRAM traffic from an ncu capture of the same
+kernel source), `cpu_baseline` (the fp64 CPU oracle on whole query rows of every pass
+of the step, rank 0 at N=1), `clocks` (NVML samples taken during the timed region),
+`extra` (the small workloads, the head-dimension, decode, prefill, row-softmax and
+GEMM workloads, timed the same way outside the timed region) and `runs` (the six
+headline runs C1, C2 non-causal / causal, C3, C4, C5 with their fraction of the peak).
 """
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -41,13 +50,24 @@ if ROOT not in sys.path:
 from workloads import WORKLOADS, make_inputs  # noqa: E402
 
 FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 * 10 ** 6
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
-# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture of
-# the same kernel build (profiles/attn_fwd_kernel_D64_f16_B4H16S1024_bench_workload.md);
-# a workload without a matching capture reports null.
-NCU_TRAFFIC_BYTES = {"C2-noncausal": 25225472}
 
+# The benchmark step: the three large workloads, one pass each.
+STEP = (("C3", True), ("C4", False), ("C5", True))
+
+# Kernel sources whose DRAM traffic the ncu figures below describe; a figure is
+# reported only while the hash of these files is the one it was captured with.
+KERNEL_SOURCES = ("attention_forward_18_b200/csrc/attn_fwd_kernel.cuh",
+                  "attention_forward_18_b200/csrc/attn_fwd.cu",
+                  "attention_forward_18_b200/csrc/ptx.cuh")
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch (ncu, --clock-control none)
+NCU_TRAFFIC = {}
+
+# North-star fractions of the dense bf16 peak per run (none stated for C1 and C2
+# non-causal).
+TARGETS = {"C2-causal": 0.50, "C3-causal": 0.50, "C4-noncausal": 0.60, "C5-causal": 0.50}
 
 # The metric both arms report (the headline benchmark's own wording).
 METRIC = "attention fwd TFLOP/s on 1 B200 (causal & non-causal), % of bf16 TC peak"
@@ -56,14 +76,16 @@ METRIC = "attention fwd TFLOP/s on 1 B200 (causal & non-causal), % of bf16 TC pe
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", default="C2", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="step", choices=["step"] + sorted(WORKLOADS))
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=1024,
+                    help="reference arm: query rows of each pass per step")
     ap.add_argument("--profile-once", action="store_true",
                     help="launch each pass of the workload once and exit (for ncu captures)")
     ap.add_argument("--profile-extra", default=None,
@@ -71,6 +93,35 @@ def parse():
                          "optionally scaled down as NAME:n (M for GEMM*, rows for SMX*, B for "
                          "DEC*, H for WD*)")
     return ap.parse_args()
+
+
+def step_passes(name):
+    """(workload, causal) of every pass of a step."""
+    if name == "step":
+        return [(WORKLOADS[n], c) for n, c in STEP]
+    w = WORKLOADS[name]
+    return [(w, c) for c in w.causal]
+
+
+def step_name(name):
+    return "+".join(w.name for w, _ in step_passes(name)) if name == "step" else name
+
+
+def pass_key(w, causal):
+    return f"{w.name}-{'causal' if causal else 'noncausal'}"
+
+
+def qkv_bytes(w):
+    """Bytes of Q, K and V of a workload (16-bit)."""
+    return 2 * w.B * w.D * (w.H * w.Sq + 2 * w.kv_heads * w.Sk)
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------- process group
@@ -119,6 +170,13 @@ def measured_peaks():
         return d, "measured"
     except (OSError, ValueError):
         return {"bf16_tflops": FALLBACK_BF16_TFLOPS, "hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def tensor_peak():
+    """The dense bf16 peak (burst figure: every timed launch here lasts about a
+    millisecond at most) and where it comes from; fp16 has the same nominal rate."""
+    peaks, kind = measured_peaks()
+    return float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), f"{kind} dense bf16 burst"
 
 
 class ClockSampler:
@@ -187,10 +245,22 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CUDA arm
+def make_flush(dev, kind):
+    """A callable that evicts L2 between timed launches: "read" sums a 256 MB buffer (L2
+    is left holding clean lines of it), "write" adds one to every element (L2 is left
+    holding dirty lines, which drain to HBM while the next launch runs)."""
+    buf = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    acc = torch.zeros((), dtype=torch.float32, device=dev)
+    if kind == "read":
+        return lambda: torch.sum(buf, 0, out=acc)
+    return lambda: buf.add_(1)
+
+
 def time_steps(launches, steps, warmup, flush, stream):
     """Run `warmup` untimed steps, then `steps` timed ones.  `launches` is a list of
-    zero-argument callables, one per kernel launch of a step.  Returns per-launch
-    event times (ms), shape [steps][len(launches)]."""
+    zero-argument callables, one per kernel launch of a step; `flush` (or None) runs
+    before each timed step, outside the events.  Returns per-launch event times (ms),
+    shape [steps][len(launches)]."""
     for _ in range(warmup):
         for f in launches:
             f()
@@ -198,7 +268,8 @@ def time_steps(launches, steps, warmup, flush, stream):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
     torch.cuda.synchronize()
     for i in range(steps):
-        flush.add_(1)  # write > L2 between timed steps
+        if flush is not None:
+            flush()
         ev[i][0].record(stream)
         for j, f in enumerate(launches):
             f()
@@ -210,18 +281,23 @@ def time_steps(launches, steps, warmup, flush, stream):
 def cuda_arm(args, world, rank, local):
     import attention_forward_18_b200 as af
 
-    w = WORKLOADS[args.workload]
+    passes = step_passes(args.workload)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
-    q, k, v = make_inputs(w)
-    dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
-    outs = {c: (torch.empty_like(dq), torch.empty((w.B, w.H, w.Sq), dtype=torch.float32,
-                                                  device=dev)) for c in w.causal}
-    dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
+    host, devt = {}, {}
+    for w, _ in passes:
+        if w.name not in host:
+            host[w.name] = make_inputs(w)
+            devt[w.name] = tuple(t.to(dev) for t in host[w.name])
+    outs = [(torch.empty_like(devt[w.name][0]),
+             torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)) for w, _ in passes]
 
-    def launcher(causal):
-        o, lse = outs[causal]
+    def launcher(i):
+        w, causal = passes[i]
+        dq, dk, dv = devt[w.name]
+        o, lse = outs[i]
+        dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
         args_ = (dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), o.data_ptr(), lse.data_ptr(),
                  w.B, w.H, w.Sq, w.Sk, w.D, int(causal), w.scale, dcode, sptr)
 
@@ -231,9 +307,10 @@ def cuda_arm(args, world, rank, local):
                 raise af.AttnError(rc, "attn_fwd")
         return f
 
-    launches = [launcher(c) for c in w.causal]
-    flops_step = sum(w.flops(c) for c in w.causal)
-    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    launches = [launcher(i) for i in range(len(passes))]
+    flops_step = sum(w.flops(c) for w, c in passes)
+    cold_inputs = all(qkv_bytes(w) > L2_BYTES for w, _ in passes)
+    flush = None if cold_inputs else make_flush(dev, "read")
 
     # bring the clocks up before the warm-up steps (untimed)
     t_end = time.perf_counter() + 0.3
@@ -259,25 +336,36 @@ def cuda_arm(args, world, rank, local):
     total_ms = max_over_ranks(total_ms, world)
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
 
-    # dominant kernel: the launch slot with the largest summed time
-    per_slot = [sum(t[j] for t in times) for j in range(len(launches))]
+    peak, peak_kind = tensor_peak()
+    per_slot = [sum(t[j] for t in times) / args.steps for j in range(len(launches))]
+    per_pass = {}
+    for j, (w, c) in enumerate(passes):
+        tf = w.flops(c) / (per_slot[j] * 1e-3) / 1e12
+        per_pass[pass_key(w, c)] = {"ms": round(per_slot[j], 5), "TFLOP/s": round(tf, 1),
+                                    "frac_of_peak": round(tf / peak, 4)}
+    # dominant kernel: the launch slot with the largest time
     dom = max(range(len(launches)), key=lambda j: per_slot[j])
-    dom_causal = w.causal[dom]
-    dom_ms = per_slot[dom] / args.steps
-    peaks, peak_kind = measured_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))  # fp16 = bf16 nominal rate
-    achieved = w.flops(dom_causal) / (dom_ms * 1e-3) / 1e12
-    key = f"{w.name}-{'causal' if dom_causal else 'noncausal'}"
+    dw, dc = passes[dom]
+    dom_ms = per_slot[dom]
+    achieved = dw.flops(dc) / (dom_ms * 1e-3) / 1e12
+    key = pass_key(dw, dc)
+    sha = kernel_source_sha()
+    cap = NCU_TRAFFIC.get(key)
+    traffic = cap["bytes"] if cap and cap["src_sha"] == sha else None
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": NCU_TRAFFIC_BYTES.get(key),
-                "kernel": f"attn_fwd_kernel<D={w.D},{w.dtype},causal={dom_causal}>",
-                "peak_source": f"{peak_kind} dense bf16 (burst; fp16 has the same nominal rate)",
+                "traffic": traffic,
+                "kernel": f"attn_fwd_kernel<D={dw.D},{dw.dtype},causal={dc}> on {key}",
+                "peak_source": f"{peak_kind} (fp16 has the same nominal rate)",
                 "per_launch_ms": round(dom_ms, 5),
-                "hbm_gbs_at_algorithmic_bytes": round(
-                    w.io_bytes() / (dom_ms * 1e-3) / 1e9, 1)}
+                "algorithmic_bytes": dw.io_bytes(),
+                "hbm_gbs_at_algorithmic_bytes": round(dw.io_bytes() / (dom_ms * 1e-3) / 1e9, 1),
+                "traffic_note": (cap["note"] if cap and traffic is not None else
+                                 "no ncu capture of this kernel source"),
+                "kernel_source_sha": sha,
+                "per_pass": per_pass}
 
-    e2e = e2e_arm(af, w, q, k, v, dev, sptr, args, world)
+    e2e = e2e_arm(af, passes, host, dev, sptr, args, world)
     clocks = sampler.summary()
 
     line = {
@@ -285,15 +373,18 @@ def cuda_arm(args, world, rank, local):
         "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16" if w.dtype == "f16" else "bf16", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} Sq={w.Sq} Sk={w.Sk} D={w.D} "
-                               f"{w.dtype}, non-causal + causal passes per step, seed {w.seed}",
-                   "B": w.B, "H": w.H, "Sq": w.Sq, "Sk": w.Sk, "D": w.D,
-                   "causal_modes": list(w.causal), "accumulate": "fp32",
-                   "l2": "flushed between timed steps (256 MB write)",
+        "dtype": "f16" if passes[0][0].dtype == "f16" else "bf16", "data": "synthetic",
+        "config": {"workload": "; ".join(
+                       f"{w.name} {'causal' if c else 'non-causal'}: B={w.B} H={w.H} Sq={w.Sq} "
+                       f"Sk={w.Sk} D={w.D} {w.dtype} seed {w.seed}"
+                       + (f" K x{w.k_scale:g}" if w.k_scale != 1.0 else "")
+                       for w, c in passes),
+                   "passes_per_step": [pass_key(w, c) for w, c in passes],
+                   "accumulate": "fp32",
+                   "l2": ("inputs larger than L2 (every pass reads >= 201 MB of Q/K/V); "
+                          "no flush" if cold_inputs else
+                          "256 MB read between timed steps (inputs fit in L2)"),
                    "parallelism": f"dp{world} (independent copy per GPU)"},
-        "per_pass_ms": {("causal" if c else "noncausal"): round(per_slot[j] / args.steps, 5)
-                        for j, c in enumerate(w.causal)},
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": len(launches) * args.steps,
@@ -302,28 +393,37 @@ def cuda_arm(args, world, rank, local):
     return line
 
 
-def e2e_arm(af, w, q, k, v, dev, sptr, args, world):
-    """Same steps through attn_fwd_host: pinned host inputs copied in, outputs copied
-    out, every step (copies inside the timed region)."""
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    oh = {c: torch.empty_like(q).pin_memory() for c in w.causal}
-    lh = {c: torch.empty((w.B, w.H, w.Sq), dtype=torch.float32).pin_memory() for c in w.causal}
-    staging = (torch.empty_like(q, device=dev), torch.empty_like(k, device=dev),
-               torch.empty_like(v, device=dev), torch.empty_like(q, device=dev),
-               torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev))
-    dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
+def e2e_arm(af, passes, host, dev, sptr, args, world):
+    """The same step through attn_fwd_host: every pass copies its workload's Q, K, V in
+    from pinned host buffers and its O and LSE out, every step (copies inside the
+    timed region)."""
+    pinned = {name: tuple(t.pin_memory() for t in qkv) for name, qkv in host.items()}
+    staging = {name: tuple(torch.empty_like(t, device=dev) for t in qkv)
+               for name, qkv in host.items()}
+    calls, h2d, d2h = [], 0, 0
+    for w, c in passes:
+        qh, kh, vh = pinned[w.name]
+        oh = torch.empty_like(qh).pin_memory()
+        lh = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32).pin_memory()
+        qd, kd, vd = staging[w.name]
+        od = torch.empty_like(qd)
+        ld = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+        dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
+        calls.append((qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(), lh.data_ptr(),
+                      qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr(),
+                      w.B, w.H, w.Sq, w.Sk, w.D, int(c), w.scale, dcode, sptr))
+        h2d += qh.nbytes + kh.nbytes + vh.nbytes
+        d2h += oh.nbytes + lh.nbytes
+        staging.setdefault("_keep", []).extend([oh, lh, od, ld])
 
     def step():
-        for c in w.causal:
-            rc = af.attn_fwd_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(),
-                                  oh[c].data_ptr(), lh[c].data_ptr(),
-                                  *(t.data_ptr() for t in staging), w.B, w.H, w.Sq, w.Sk,
-                                  w.D, int(c), w.scale, dcode, sptr)
+        for a in calls:
+            rc = af.attn_fwd_host(*a)
             if rc != 0:
                 raise af.AttnError(rc, "attn_fwd_host")
 
-    steps = max(3, min(args.steps, 50))
-    for _ in range(max(3, args.warmup // 4)):
+    steps = max(3, min(args.steps, 20))
+    for _ in range(3):
         step()
     barrier(world)
     torch.cuda.synchronize()
@@ -336,24 +436,27 @@ def e2e_arm(af, w, q, k, v, dev, sptr, args, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    flops_step = sum(w.flops(c) for c in w.causal)
-    n = len(w.causal)
+    flops_step = sum(w.flops(c) for w, c in passes)
+    shared = len({w.name for w, _ in passes}) < len(passes)
     return {"value": round(world * flops_step * steps / (ms * 1e-3) / 1e12, 4),
             "unit": "TFLOP/s", "steps": steps,
-            "h2d_bytes_per_step": n * (q.nbytes + k.nbytes + v.nbytes),
-            "d2h_bytes_per_step": n * (q.nbytes + 4 * w.B * w.H * w.Sq),
-            "path": "attn_fwd_host (pinned host buffers, copies + kernel on one stream)"}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "path": "attn_fwd_host per pass (pinned host buffers, copies + kernel on one "
+                    "stream)" + ("; passes on the same tensors each copy them in"
+                                 if shared else "")}
 
 
 def extra_workloads(af_names, world):
-    """Other workloads, timed the same way (cold L2 between launches), one line each."""
+    """Other workloads, one launch per pass timed like the step (median of 20), with a
+    256 MB read between launches so a workload whose inputs fit in L2 starts cold; for
+    those small workloads the same with a 256 MB write between launches (the dirty lines
+    drain while the next launch runs) is reported beside it."""
     import attention_forward_18_b200 as af
+    from workloads import WIDE_WORKLOADS
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
-    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    peaks, peak_kind = measured_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
-    from workloads import WIDE_WORKLOADS
+    flush_read, flush_write = make_flush(dev, "read"), make_flush(dev, "write")
+    peak, peak_kind = tensor_peak()
     res = {}
     for name in af_names:
         w = WORKLOADS[name] if name in WORKLOADS else WIDE_WORKLOADS[name]
@@ -368,20 +471,24 @@ def extra_workloads(af_names, world):
                                  dcode, stream.cuda_stream)
                 if rc != 0:
                     raise af.AttnError(rc, "attn_fwd")
-            t = time_steps([f], 20, 5, flush, stream)
-            ms = statistics.median(x[0] for x in t)
+            ms = statistics.median(x[0] for x in time_steps([f], 20, 5, flush_read, stream))
             tf = w.flops(c) / (ms * 1e-3) / 1e12
-            res[f"{name}{'-causal' if c else ''}"] = {
-                "shape": f"B={w.B} H={w.H} S={w.Sq} D={w.D} {w.dtype}",
-                "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
-                "frac_of_peak": round(tf / peak, 4),
-                "hbm_gbs_at_algorithmic_bytes": round(w.io_bytes() / (ms * 1e-3) / 1e9, 1)}
+            entry = {"shape": f"B={w.B} H={w.H} S={w.Sq} D={w.D} {w.dtype}",
+                     "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                     "frac_of_peak": round(tf / peak, 4),
+                     "hbm_gbs_at_algorithmic_bytes": round(w.io_bytes() / (ms * 1e-3) / 1e9, 1)}
+            if qkv_bytes(w) < L2_BYTES:
+                ms_w = statistics.median(
+                    x[0] for x in time_steps([f], 20, 5, flush_write, stream))
+                entry["ms_write_flush"] = round(ms_w, 4)
+                entry["TFLOP/s_write_flush"] = round(w.flops(c) / (ms_w * 1e-3) / 1e12, 1)
+            res[pass_key(w, c)] = entry
         status = af.attn_fwd_status(stream)
         if status != 0:
             raise af.AttnError(status, f"device status after {name}")
         del q, k, v, o, lse
         torch.cuda.empty_cache()
-    res["peak_TFLOP/s"] = f"{peak} ({peak_kind} dense bf16 burst)"
+    res["peak_TFLOP/s"] = f"{peak} ({peak_kind})"
     return res
 
 
@@ -391,8 +498,7 @@ def graph_launches(names, reps=20):
     in L2 after the first launch -- stated in the line)."""
     import attention_forward_18_b200 as af
     dev = torch.device("cuda", torch.cuda.current_device())
-    peaks, _ = measured_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    peak, _ = tensor_peak()
     res = {}
     stream = torch.cuda.Stream(dev)
     for name in names:
@@ -427,7 +533,7 @@ def graph_launches(names, reps=20):
                     times.append(e0.elapsed_time(e1) / reps)
             ms = statistics.median(times)
             tf = w.flops(c) / (ms * 1e-3) / 1e12
-            res[f"{name}{'-causal' if c else ''}"] = {
+            res[pass_key(w, c)] = {
                 "ms_per_launch": round(ms, 5), "TFLOP/s": round(tf, 1),
                 "frac_of_peak": round(tf / peak, 4),
                 "note": f"{reps} launches per graph replay, L2 warm"}
@@ -446,7 +552,7 @@ def decode_workloads(names):
     from workloads import DECODE_WORKLOADS
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
-    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = make_flush(dev, "read")
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     res = {}
@@ -497,9 +603,8 @@ def prefill_workloads(names):
     from workloads import PREFILL_WORKLOADS, visible_pairs
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
-    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    peaks, peak_kind = measured_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    flush = make_flush(dev, "read")
+    peak, peak_kind = tensor_peak()
     res = {}
     for name in names:
         w = PREFILL_WORKLOADS[name]
@@ -527,7 +632,7 @@ def prefill_workloads(names):
             raise af.AttnError(status, f"device status after {name}")
         del q, k, v, o, lse
         torch.cuda.empty_cache()
-    res["peak_TFLOP/s"] = f"{peak} ({peak_kind} dense bf16 burst)"
+    res["peak_TFLOP/s"] = f"{peak} ({peak_kind})"
     return res
 
 
@@ -538,7 +643,7 @@ def softmax_workloads(names):
     from workloads import SOFTMAX_WORKLOADS, make_rows
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
-    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = make_flush(dev, "read")
     peaks, peak_kind = measured_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     codes = {"f16": af.ATTN_F16, "bf16": af.ATTN_BF16, "f32": af.SOFTMAX_F32}
@@ -571,9 +676,8 @@ def gemm_workloads(names):
     from workloads import GEMM_WORKLOADS, make_gemm
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
-    flush = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    peaks, peak_kind = measured_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+    flush = make_flush(dev, "read")
+    peak, peak_kind = tensor_peak()
     res = {}
     for name in names:
         g = GEMM_WORKLOADS[name]
@@ -606,60 +710,85 @@ def gemm_workloads(names):
             raise af.AttnError(status, f"device status after {name}")
         del a, w, b, c
         torch.cuda.empty_cache()
-    res["peak_TFLOP/s"] = f"{peak} ({peak_kind} dense bf16 burst)"
+    res["peak_TFLOP/s"] = f"{peak} ({peak_kind})"
     return res
 
 
 # ---------------------------------------------------------------- oracle (CPU) arm
-def oracle_sample(w, seconds, max_heads=None):
-    """Time the fp64 CPU oracle as it stands on whole heads of the workload (every
-    causal mode of the step), adding heads until `seconds` have passed or the
-    workload is exhausted.  Returns (TFLOP/s, cores, description)."""
+def oracle_inputs(passes):
+    """fp64 numpy copies of every workload's inputs (the 16-bit values upcast exactly,
+    as the oracle reads them)."""
+    out = {}
+    for w, _ in passes:
+        if w.name not in out:
+            q, k, v = make_inputs(w)
+            out[w.name] = (q.double().numpy(), k.double().numpy(), v.double().numpy())
+    return out
+
+
+def oracle_rows_timed(passes, inputs, rows_per_pass, rng):
+    """One sample: `rows_per_pass` whole query rows (uniform over batch, head and row)
+    of every pass through the oracle's row entry point, which materialises each row's
+    Sk scores in fp64, masks them, takes the softmax and multiplies by V.  Returns the
+    FLOPs the metric counts for those rows (4*Sk*D a row, halved for causal) and the
+    oracle's time."""
+    import numpy as np
     import oracle
-    q, k, v = make_inputs(w)
-    qd = q.double().numpy().reshape(w.B * w.H, 1, w.Sq, w.D)
-    kd = k.double().numpy().reshape(w.B * w.H, 1, w.Sk, w.D)
-    vd = v.double().numpy().reshape(w.B * w.H, 1, w.Sk, w.D)
-    threads = oracle.num_threads()
-    total_heads = w.B * w.H if max_heads is None else min(max_heads, w.B * w.H)
-    chunk = max(1, threads)
-    done, flops, t_used = 0, 0.0, 0.0
-    while done < total_heads and (done == 0 or t_used < seconds):
-        n = min(chunk, total_heads - done)
-        sl = slice(done, done + n)
-        qs = qd[sl].reshape(1, n, w.Sq, w.D)
-        ks = kd[sl].reshape(1, n, w.Sk, w.D)
-        vs = vd[sl].reshape(1, n, w.Sk, w.D)
+    flops, secs = 0.0, 0.0
+    for w, c in passes:
+        qd, kd, vd = inputs[w.name]
+        rows = np.stack([rng.integers(0, w.B, rows_per_pass), rng.integers(0, w.H, rows_per_pass),
+                         rng.integers(0, w.Sq, rows_per_pass)], axis=1)
+        rows = rows[np.lexsort((rows[:, 2], rows[:, 1], rows[:, 0]))]  # head by head
         t0 = time.perf_counter()
-        for c in w.causal:
-            oracle.attn_ref(qs, ks, vs, c, w.scale)
-        t_used += time.perf_counter() - t0
-        flops += sum(4.0 * n * w.Sq * w.Sk * w.D * (0.5 if c else 1.0) for c in w.causal)
-        done += n
-    desc = (f"{done} of {w.B * w.H} heads of {w.name} (both passes of the step), "
-            f"{t_used:.1f} s of oracle time")
-    return flops / t_used / 1e12, threads, desc
+        oracle.attn_ref_rows(qd, kd, vd, rows, c, w.scale)
+        secs += time.perf_counter() - t0
+        flops += rows_per_pass * 4.0 * w.Sk * w.D * (0.5 if c else 1.0)
+    return flops, secs
+
+
+def oracle_sample(passes, seconds):
+    """Time the fp64 CPU oracle as it stands on whole query rows of every pass of the
+    step, a chunk of rows of each pass in turn, until `seconds` of oracle time have
+    passed.  Returns (TFLOP/s, cores, description)."""
+    import numpy as np
+    import oracle
+    inputs = oracle_inputs(passes)
+    rng = np.random.default_rng(2024)
+    threads = oracle.num_threads()
+    chunk = max(64, 16 * threads)
+    flops, secs, rows = 0.0, 0.0, 0
+    while rows == 0 or secs < seconds:
+        f, s = oracle_rows_timed(passes, inputs, chunk, rng)
+        flops += f
+        secs += s
+        rows += chunk
+    desc = (f"{rows} whole query rows of each of "
+            f"{', '.join(pass_key(w, c) for w, c in passes)} (uniform over batch, head and "
+            f"row; the oracle's row entry point), {secs:.1f} s of oracle time")
+    return flops / secs / 1e12, threads, desc
 
 
 def reference_arm(args, world, rank):
     """The oracle as the reference implementation: K timed steps, each a bounded
-    sample (whole heads) of the workload, on this host's cores."""
-    w = WORKLOADS[args.workload]
+    sample (whole query rows of every pass of the step) on this host's cores."""
+    import numpy as np
     import oracle
+    passes = step_passes(args.workload)
+    inputs = oracle_inputs(passes)
+    rng = np.random.default_rng(2025)
     threads = oracle.num_threads()
-    per_step_heads = max(1, threads)
     for _ in range(args.warmup):
-        oracle_sample(w, 0.0, max_heads=per_step_heads)
+        oracle_rows_timed(passes, inputs, args.ref_rows, rng)
     t_flops, t_time = 0.0, 0.0
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        tf, cores, desc = oracle_sample(w, 0.0, max_heads=per_step_heads)
-        dt = time.perf_counter() - t0
-        t_time += dt
-        t_flops += tf * 1e12 * dt
+        f, s = oracle_rows_timed(passes, inputs, args.ref_rows, rng)
+        t_flops += f
+        t_time += s
     value = t_flops / t_time / 1e12
-    sample = (f"per step: {per_step_heads} whole heads of {w.name} "
-              f"(B={w.B} H={w.H} S={w.Sq} D={w.D}), non-causal + causal")
+    sample = (f"per step: {args.ref_rows} whole query rows of each of "
+              f"{', '.join(pass_key(w, c) for w, c in passes)} (uniform over batch, head "
+              f"and row)")
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -667,8 +796,11 @@ def reference_arm(args, world, rank):
         "warmup": args.warmup, "ms_per_step": round(t_time / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} Sq={w.Sq} Sk={w.Sk} D={w.D} "
-                               f"{w.dtype} inputs upcast to fp64, non-causal + causal",
+        "config": {"workload": f"{step_name(args.workload)}: "
+                               + "; ".join(f"{w.name} {'causal' if c else 'non-causal'} "
+                                           f"B={w.B} H={w.H} Sq={w.Sq} Sk={w.Sk} D={w.D} "
+                                           f"{w.dtype}" for w, c in passes)
+                               + "; inputs upcast to fp64",
                    "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
@@ -677,21 +809,43 @@ def reference_arm(args, world, rank):
     }
 
 
+def runs_summary(line):
+    """The six headline runs (C1, C2 non-causal and causal, C3, C4, C5): TFLOP/s and
+    fraction of the dense bf16 peak, with the stated target where there is one."""
+    out = {}
+    extra = line.get("extra", {})
+    found = dict(extra.items())
+    found.update(line["roofline"]["per_pass"])
+    for key in ("C1-noncausal", "C2-noncausal", "C2-causal", "C3-causal", "C4-noncausal",
+                "C5-causal"):
+        r = found.get(key)
+        if not isinstance(r, dict) or "TFLOP/s" not in r:
+            continue
+        e = {"TFLOP/s": r["TFLOP/s"], "frac": r["frac_of_peak"]}
+        if key in TARGETS:
+            e["target"] = TARGETS[key]
+        out[key] = e
+    return out
+
+
 def profile_once(args):
     """One launch per pass of the workload, nothing else on the GPU before it except
     the input copies (a short, self-ending command for ncu)."""
     import attention_forward_18_b200 as af
     if args.profile_extra:
         return profile_extra(args.profile_extra)
-    w = WORKLOADS[args.workload]
-    q, k, v = (t.cuda() for t in make_inputs(w))
-    for c in w.causal:
+    passes = step_passes(args.workload)
+    inputs = {}
+    for w, c in passes:
+        if w.name not in inputs:
+            inputs[w.name] = tuple(t.cuda() for t in make_inputs(w))
+        q, k, v = inputs[w.name]
         af.attention(q, k, v, causal=c, scale=w.scale)
     torch.cuda.synchronize()
     status = af.attn_fwd_status()
     if status != 0:
         raise af.AttnError(status, "device status")
-    print(json.dumps({"profile_once": w.name, "passes": list(w.causal)}))
+    print(json.dumps({"profile_once": [pass_key(w, c) for w, c in passes]}))
 
 
 def profile_extra(spec):
@@ -755,7 +909,8 @@ def main():
         # the other workloads once, on a single-GPU run (a multi-GPU run would hold every
         # GPU while rank 0 alone works through them)
         if rank == 0 and world == 1 and not args.no_extra:
-            line["extra"] = extra_workloads(["C3", "C4", "C5", "WD192", "WD256"], world)
+            small = [n for n in ("C1", "C2") if n != args.workload]
+            line["extra"] = extra_workloads(small + ["WD192", "WD256"], world)
             line["extra"]["cuda_graph"] = graph_launches(["C1", "C2"])
             line["extra"]["decode_splitkv"] = decode_workloads(
                 ["DEC1", "DEC2", "DEC3", "DEC4", "DEC5", "DEC6"])
@@ -763,10 +918,10 @@ def main():
             line["extra"]["row_softmax"] = softmax_workloads(["SMX1", "SMX2", "SMX3"])
             line["extra"]["gemm_bias_act"] = gemm_workloads(["GEMM1", "GEMM2", "GEMM3"])
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            w = WORKLOADS[args.workload]
-            tf, cores, desc = oracle_sample(w, args.cpu_seconds)
+            tf, cores, desc = oracle_sample(step_passes(args.workload), args.cpu_seconds)
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores,
                                     "kind": "oracle", "sample": desc}
+        line["runs"] = runs_summary(line)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

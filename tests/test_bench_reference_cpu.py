@@ -24,7 +24,7 @@ def test_reference_arm_json_line():
     assert line["metric"] == bench.METRIC
     assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
     assert line["value"] > 0 and line["steps"] == 1 and line["n_gpus"] == 1
-    assert line["config"]["workload"].startswith("C2:")
+    assert line["config"]["workload"].startswith("C3+C4+C5:")
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
     e2e = line["e2e"]
