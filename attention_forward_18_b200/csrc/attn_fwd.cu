@@ -28,6 +28,9 @@ constexpr int kMaxSeq = 1 << 24;
 constexpr int kMaxHeads = 1 << 24;
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 1024;
+// Causal unit order: K/V bytes of the heads whose units run at the same time, kept to
+// this part of the 126 MB L2 (the rest holds Q tiles and outputs on their way out).
+constexpr int64_t kCausalGroupKvBytes = 48ll << 20;
 
 // cuTensorMapEncodeTiled, fetched through the runtime so the library needs no
 // link against libcuda.
@@ -96,8 +99,9 @@ bool encode_chunked_map(CUtensorMap* m, const void* base, int D, int S, int BH, 
     return r == CUDA_SUCCESS;
 }
 
-// Per-device facts checked once: compute capability 10.x and the SM count (the
-// persistent grid has one CTA per SM).
+// Per-device facts checked once: compute capability 10.0 and the SM count (the
+// persistent grid has one CTA per SM).  Kept for the life of the process (not valid
+// across cudaDeviceReset, like the other per-device set-up below).
 int check_device(int* num_sms) {
     static int dev_ok[kMaxDevices];  // 0 unknown, 1 ok, -1 not sm_100
     static int sms[kMaxDevices];
@@ -109,13 +113,15 @@ int check_device(int* num_sms) {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (dev_ok[dev] == 0) {
-        int major = 0, count = 0;
+        int major = 0, minor = 0, count = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
             return ATTN_ERR_DEVICE;
         }
-        dev_ok[dev] = (major == 10 && count > 0) ? 1 : -1;
+        // the library carries sm_100a code only, which no other 10.x part runs
+        dev_ok[dev] = (major == 10 && minor == 0 && count > 0) ? 1 : -1;
         sms[dev] = count;
     }
     if (num_sms) *num_sms = sms[dev];
@@ -419,6 +425,9 @@ int launch_merge(const float* ws_o, const float* ws_lse, void* o, float* lse, in
 // n_splits == 0: the whole pass (16-bit O and LSE written by the attention kernel);
 // n_splits >= 1: a split pass through `workspace`, then the merge kernel.
 // Hkv: K/V heads (divides H); mask: ATTN_MASK_*.
+// Host-side debug flag of attn_fwd_debug: report a failed TMA descriptor encoding.
+constexpr unsigned kFlagFailTensorMap = 2u;
+
 int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
         int Sq, int Sk, int D, int mask, float scale, int dtype, cudaStream_t stream,
         unsigned flags, int n_splits = 0, void* workspace = nullptr, size_t workspace_bytes = 0) {
@@ -459,6 +468,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int kv_keys = wide ? attn::wide::WBN : attn::BN;
     const int q_units = wide ? attn::wide::WBM : attn::ROWS_PER_CTA;
     CUtensorMap tq, tk, tv;
+    if (flags & kFlagFailTensorMap) return ATTN_ERR_TENSORMAP;
     if (pair_path) {
         // one box per half tile: Q 128 rows and K 64 keys, all 64-column chunks; V 128
         // keys, this CTA's D/2 columns (64-column chunks at D = 256, 32-column at 192)
@@ -487,6 +497,11 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int n_kv = (Sk + kv_keys - 1) / kv_keys;
     p.n_splits = n_splits > 0 ? n_splits : 1;
     p.chunk_tiles = (n_kv + p.n_splits - 1) / p.n_splits;
+    {
+        const int64_t kv_head_bytes = static_cast<int64_t>(4) * Sk * D;  // K and V, 16-bit
+        const int64_t g = kCausalGroupKvBytes / kv_head_bytes;
+        p.head_group = static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
+    }
     p.ws_o = n_splits > 0 ? static_cast<float*>(workspace) : nullptr;
     p.ws_lse = n_splits > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                        ws_o_bytes(B, H, Sq, D, n_splits))
@@ -496,7 +511,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     // nonzero multiplier to keep masked scores at -inf (not -inf * 0 = NaN), and with
     // 1e-30 every visible weight is 2^(~1e-28) = 1.0f exactly.
     if (p.scale_log2 == 0.f) p.scale_log2 = 1e-30f;
-    p.flags = flags;
+    p.flags = flags & attn::FLAG_SKIP_Q_LOAD;
     // persistent: one CTA per SM (at most one per work unit), each walking its units
     const int64_t n_units = static_cast<int64_t>(p.n_qp) * BH * p.n_splits;
     if (n_units > INT_MAX) return ATTN_ERR_SHAPE;
@@ -556,7 +571,8 @@ int attn_fwd_debug(const void* q, const void* k, const void* v, void* o, float* 
                    int H, int Sq, int Sk, int D, int causal, float scale, int dtype,
                    attn_stream_t stream, unsigned flags) {
     return run(q, k, v, o, lse, B, H, H, Sq, Sk, D, mask_of(causal), scale, dtype,
-               reinterpret_cast<cudaStream_t>(stream), flags & attn::FLAG_SKIP_Q_LOAD);
+               reinterpret_cast<cudaStream_t>(stream),
+               flags & (attn::FLAG_SKIP_Q_LOAD | kFlagFailTensorMap));
 }
 
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,

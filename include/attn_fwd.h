@@ -183,6 +183,10 @@ int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal);
  *   One scratch per device: calls on one device that can overlap (different streams,
  *   or threads without ordering) race on it and give undefined results.  Calls
  *   ordered on one stream are safe.
+ *   The looked-up address (like the library's other per-device set-up: kernel
+ *   attributes, cluster occupancy) is kept for the life of the process and is not
+ *   valid across cudaDeviceReset: a process that resets a device must not call this
+ *   library on that device again.
  */
 int attn_fwd_splitkv_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
                              int B, int H, int Sq, int Sk, int D, int causal, float scale,
@@ -203,9 +207,11 @@ const char *attn_fwd_strerror(int code);
 int attn_fwd_abi_version(void);
 
 /*
- * attn_fwd_debug -- attn_fwd with kernel debug flags, for the tests.  Flag 1 makes
- * the TMA producer skip the Q load so the MMA warp's first wait runs out: the call
- * must end with ATTN_ERR_TIMEOUT in the status word, not hang.  Flag 0 is attn_fwd.
+ * attn_fwd_debug -- attn_fwd with debug flags, for the tests.  Flag 1 makes the TMA
+ * producer skip the Q load so the MMA warp's first wait runs out: the call must end
+ * with ATTN_ERR_TIMEOUT in the status word, not hang.  Flag 2 (host side only) makes
+ * the TMA descriptor encoding report failure: the call returns ATTN_ERR_TENSORMAP
+ * and launches nothing.  Flag 0 is attn_fwd.
  */
 int attn_fwd_debug(const void *q, const void *k, const void *v, void *o, float *lse,
                    int B, int H, int Sq, int Sk, int D, int causal, float scale,

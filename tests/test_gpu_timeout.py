@@ -77,3 +77,25 @@ def test_starved_pipeline_on_the_wide_head_dimensions(D, Sq):
     o2, l2 = af.attention(q, k, v, causal=True, scale=0.07)
     torch.cuda.synchronize()
     assert af.attn_fwd_status() == 0 and torch.isfinite(o2.float()).all()
+
+
+@pytest.mark.parametrize("D,Sq", [(64, 300), (128, 300), (256, 300), (256, 64)])
+def test_failed_descriptor_encoding_returns_an_error_and_launches_nothing(D, Sq):
+    """A TMA descriptor encoding that fails (forced by the host-side debug flag 2, on
+    the D <= 128 kernel's, the CTA-pair kernel's and the wide kernel's maps) makes the
+    call return ATTN_ERR_TENSORMAP before any launch: the outputs keep their sentinel
+    values and the status word stays clear; the next normal call is unaffected."""
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, Sq, 400, D, "bf16", 26))
+    o = torch.full_like(q, 7.0)
+    lse = torch.full((1, 2, Sq), 7.0, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert af.attn_fwd_status() == 0
+    rc = af.attn_fwd_debug(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                           lse.data_ptr(), 1, 2, Sq, 400, D, 1, 0.07, af.ATTN_BF16, stream, 2)
+    assert rc == af.ATTN_ERR_TENSORMAP
+    torch.cuda.synchronize()
+    assert bool((o == 7.0).all()) and bool((lse == 7.0).all())
+    assert af.attn_fwd_status() == 0
+    o2, l2 = af.attention(q, k, v, causal=True, scale=0.07)
+    torch.cuda.synchronize()
+    assert af.attn_fwd_status() == 0 and torch.isfinite(o2.float()).all()

@@ -1,11 +1,15 @@
 """attn_fwd_splitkv_noalloc: the split-KV pass into the library's own static scratch
-instead of a caller workspace.  Compared, through the C ABI, with attn_fwd_splitkv on
-the same inputs within the parity tolerances, on two calls in a row."""
+instead of a caller workspace (for callers that cannot allocate device memory per
+call).  Compared, through the C ABI, with attn_fwd_splitkv on the same inputs and with
+the fp64 oracle, within the parity tolerances, on two calls in a row; the cases cover
+the D <= 128 kernel and, at D = 256, the wide kernel's split pass."""
+import numpy as np
 import pytest
 import torch
 
 import attention_forward_18_b200 as af
-from parity import LSE_TOL, O_TOL
+import oracle
+from parity import LSE_TOL, O_TOL, compare
 from workloads import make_qkv
 
 FAKE = 0x10000000  # 16-byte aligned fake device addresses for argument checks
@@ -49,12 +53,18 @@ def _run_both(q, k, v, causal, n, stream):
 def test_two_calls_in_a_row_match_the_workspace_entry_point():
     stream = torch.cuda.current_stream().cuda_stream
     cases = [((2, 8, 4, 5000, 128, "bf16", 31), False, 6),
-             ((3, 4, 16, 3000, 64, "f16", 32), True, 3)]
+             ((3, 4, 16, 3000, 64, "f16", 32), True, 3),
+             ((1, 4, 1, 3000, 256, "bf16", 33), False, 4)]
     for (B, H, Sq, Sk, D, dt, seed), causal, n in cases:
-        q, k, v = (t.cuda() for t in make_qkv(B, H, Sq, Sk, D, dt, seed))
+        qc, kc, vc = make_qkv(B, H, Sq, Sk, D, dt, seed)
+        o_orc, l_orc = oracle.attn_ref(qc.double().numpy(), kc.double().numpy(),
+                                       vc.double().numpy(), causal, D ** -0.5)
+        q, k, v = (t.cuda() for t in (qc, kc, vc))
         o, lse, o_ref, l_ref = _run_both(q, k, v, causal, n, stream)
         torch.cuda.synchronize()
         assert af.attn_fwd_status() == 0
         assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
         assert (o.float() - o_ref.float()).abs().max().item() <= O_TOL
         assert (lse - l_ref).abs().max().item() <= LSE_TOL
+        compare(o.double().cpu().numpy(), lse.double().cpu().numpy(), o_orc, l_orc,
+                f"noalloc B{B} H{H} Sq{Sq} Sk{Sk} D{D} splits {n}")
