@@ -75,13 +75,13 @@ _lib.attn_fwd_splitkv.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _i, _i, _vp, ctypes
 _lib.attn_fwd_splitkv.restype = _i
 _lib.attn_fwd_splitkv_workspace_bytes.argtypes = [_i] * 5
 _lib.attn_fwd_splitkv_workspace_bytes.restype = ctypes.c_size_t
-_lib.attn_fwd_splitkv_default_splits.argtypes = [_i] * 5
+_lib.attn_fwd_splitkv_default_splits.argtypes = [_i] * 6
 _lib.attn_fwd_splitkv_default_splits.restype = _i
 _lib.attn_fwd_splitkv_noalloc.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _i, _i, _vp]
 _lib.attn_fwd_splitkv_noalloc.restype = _i
 _lib.attn_fwd_ex.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _i, _i, _vp, ctypes.c_size_t, _vp]
 _lib.attn_fwd_ex.restype = _i
-_lib.attn_fwd_ex_default_splits.argtypes = [_i] * 6
+_lib.attn_fwd_ex_default_splits.argtypes = [_i] * 7
 _lib.attn_fwd_ex_default_splits.restype = _i
 _lib.gemm_bias_act.argtypes = [_vp] * 4 + [_i] * 5 + [_vp]
 _lib.gemm_bias_act.restype = _i
@@ -157,16 +157,16 @@ def attn_fwd_ex(q, k, v, o, lse, B, H, H_kv, Sq, Sk, D, mask, scale, dtype, n_sp
                             int(dtype), int(n_splits), workspace, int(workspace_bytes), stream)
 
 
-def ex_default_splits(B, H, H_kv, Sq, Sk, mask=ATTN_MASK_NONE):
-    return _lib.attn_fwd_ex_default_splits(B, H, H_kv, Sq, Sk, int(mask))
+def ex_default_splits(B, H, H_kv, Sq, Sk, mask=ATTN_MASK_NONE, D=128):
+    return _lib.attn_fwd_ex_default_splits(B, H, H_kv, Sq, Sk, int(D), int(mask))
 
 
 def splitkv_workspace_bytes(B, H, Sq, D, n_splits):
     return _lib.attn_fwd_splitkv_workspace_bytes(B, H, Sq, D, n_splits)
 
 
-def splitkv_default_splits(B, H, Sq, Sk, causal=False):
-    return _lib.attn_fwd_splitkv_default_splits(B, H, Sq, Sk, int(bool(causal)))
+def splitkv_default_splits(B, H, Sq, Sk, causal=False, D=128):
+    return _lib.attn_fwd_splitkv_default_splits(B, H, Sq, Sk, int(D), int(bool(causal)))
 
 
 def attn_fwd_status(stream=None):
@@ -246,7 +246,7 @@ def attention_splitkv(q, k, v, causal=False, scale=None, n_splits=None, out=None
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if n_splits is None:
-        n_splits = splitkv_default_splits(B, H, Sq, Sk, causal)
+        n_splits = splitkv_default_splits(B, H, Sq, Sk, causal, D)
     nbytes = splitkv_workspace_bytes(B, H, Sq, D, n_splits)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
@@ -275,7 +275,7 @@ def attention_ex(q, k, v, mask=ATTN_MASK_NONE, scale=None, n_splits=0, out=None,
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if n_splits is None:
-        n_splits = ex_default_splits(B, H, Hkv, Sq, Sk, mask)
+        n_splits = ex_default_splits(B, H, Hkv, Sq, Sk, mask, D)
     nbytes = splitkv_workspace_bytes(B, H, Sq, D, n_splits) if n_splits > 0 else 0
     if n_splits > 0 and workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)

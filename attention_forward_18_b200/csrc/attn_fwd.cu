@@ -28,9 +28,6 @@ constexpr int kMaxSeq = 1 << 24;
 constexpr int kMaxHeads = 1 << 24;
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 1024;
-// Causal unit order: K/V bytes of the heads whose units run at the same time, kept to
-// this part of the 126 MB L2 (the rest holds Q tiles and outputs on their way out).
-constexpr int64_t kCausalGroupKvBytes = 48ll << 20;
 
 // cuTensorMapEncodeTiled, fetched through the runtime so the library needs no
 // link against libcuda.
@@ -497,11 +494,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
     const int n_kv = (Sk + kv_keys - 1) / kv_keys;
     p.n_splits = n_splits > 0 ? n_splits : 1;
     p.chunk_tiles = (n_kv + p.n_splits - 1) / p.n_splits;
-    {
-        const int64_t kv_head_bytes = static_cast<int64_t>(4) * Sk * D;  // K and V, 16-bit
-        const int64_t g = kCausalGroupKvBytes / kv_head_bytes;
-        p.head_group = static_cast<int>(g < 1 ? 1 : g > BH ? BH : g);
-    }
+
     p.ws_o = n_splits > 0 ? static_cast<float*>(workspace) : nullptr;
     p.ws_lse = n_splits > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                                        ws_o_bytes(B, H, Sq, D, n_splits))
@@ -534,13 +527,13 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
 
 int mask_of(int causal) { return causal ? ATTN_MASK_CAUSAL : ATTN_MASK_NONE; }
 
-// Split count for `units` (query block, head) pairs over KV tiles 0..n_kv-1: persistent
-// CTAs take units round-robin, so a pass lasts about
-//   ceil(units * n / SMs) rounds x (tiles per range + a fill of ~2 tiles);
+// Split count for `units` (query block, head) pairs over KV tiles 0..n_kv-1 on `slots`
+// units that run at once (SMs, or CTA pairs): persistent CTAs take units round-robin,
+// so a pass lasts about
+//   ceil(units * n / slots) rounds x (tiles per range + a fill of ~2 tiles);
 // the n with the least of that (the fewest splits among equals: less to merge).
-int balanced_splits(int64_t units, int n_kv) {
-    int num_sms = 0;
-    if (check_device(&num_sms) != ATTN_OK) num_sms = 148;
+int balanced_splits(int64_t units, int n_kv, int slots) {
+    const int num_sms = slots;
     int best = 1;
     int64_t best_cost = INT64_MAX;
     const int n_hi = n_kv < kMaxSplits ? n_kv : kMaxSplits;
@@ -614,19 +607,28 @@ size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_split
     return ws_bytes(B, H, Sq, D, n_splits);
 }
 
-int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal) {
-    return attn_fwd_ex_default_splits(B, H, H, Sq, Sk, mask_of(causal));
+int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int D, int causal) {
+    return attn_fwd_ex_default_splits(B, H, H, Sq, Sk, D, mask_of(causal));
 }
 
-int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int mask) {
-    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Sq < 1 || Sk < 1 || mask < 0 ||
-        mask > ATTN_MASK_CAUSAL_BOTTOM_RIGHT)
+int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int D, int mask) {
+    if (B < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || Sq < 1 || Sk < 1 || !head_dim_ok(D) ||
+        mask < 0 || mask > ATTN_MASK_CAUSAL_BOTTOM_RIGHT)
         return 0;
+    int num_sms = 0;
+    if (check_device(&num_sms) != ATTN_OK) num_sms = 148;
+    // the geometry of the kernel run() picks for these sizes: D <= 128 and the CTA pairs
+    // take 256-row units and 128-key tiles (a pair's unit on two SMs); the wide kernel
+    // (D = 192 / 256, at most 128 packed rows) 128-row units and 64-key tiles
     const int64_t rows = static_cast<int64_t>(H / H_kv) * Sq;
-    const int64_t units = (rows + attn::ROWS_PER_CTA - 1) / attn::ROWS_PER_CTA * B * H_kv;
+    const bool wide = is_wide(D) && rows <= attn::BM;
+    const bool pair = is_wide(D) && !wide;
+    const int q_units = wide ? attn::wide::WBM : attn::ROWS_PER_CTA;
+    const int kv_keys = wide ? attn::wide::WBN : attn::BN;
+    const int64_t units = (rows + q_units - 1) / q_units * B * H_kv;
     // with the top-left causal mask no row sees a key past min(Sq, Sk)
     const int keys = mask == ATTN_MASK_CAUSAL ? (Sq < Sk ? Sq : Sk) : Sk;
-    return balanced_splits(units, (keys + attn::BN - 1) / attn::BN);
+    return balanced_splits(units, (keys + kv_keys - 1) / kv_keys, pair ? num_sms / 2 : num_sms);
 }
 
 int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -702,6 +704,6 @@ const char* attn_fwd_strerror(int code) {
     }
 }
 
-int attn_fwd_abi_version(void) { return 1; }
+int attn_fwd_abi_version(void) { return 2; }
 
 }  // extern "C"

@@ -89,7 +89,6 @@ struct Params {
     int causal_off;     // causal: key j visible to position i iff j <= i + causal_off
     int n_splits;       // KV ranges per (query pair, head); 1 for the whole pass
     int chunk_tiles;    // KV tiles per range
-    int head_group;     // causal unit order: heads per group (see decode_unit)
     float scale_log2;   // scale * log2(e)
     uint32_t flags;
 };
@@ -104,11 +103,10 @@ struct SmemLayout {
     static constexpr int V_OFF = K_OFF + NS * TILE_BYTES;
     static constexpr int FM_OFF = V_OFF + NS * TILE_BYTES;  // final max  float [2][128]
     static constexpr int FL_OFF = FM_OFF + 2 * BM * 4;      // final sum  float [2][128]
-    static constexpr int FR_OFF = FL_OFF + 2 * BM * 4;      // final rounded sum [2][128]
-    static constexpr int BAR_OFF = FR_OFF + 2 * BM * 4;
+    static constexpr int BAR_OFF = FL_OFF + 2 * BM * 4;
     // q_full[2], k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2],
-    // p_full[2], o_final[2], stats[2], o_free[2], q_empty, drain
-    static constexpr int NBAR = 2 + 4 * NS + 2 * 5 + 2;
+    // p_full[2], o_final[2], stats[2], o_free[2], q_empty[2], drain
+    static constexpr int NBAR = 2 + 4 * NS + 2 * 6 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // tmem base, error flag
     static constexpr int BYTES = MISC_OFF + 16;
     static constexpr int ALLOC = BYTES + 1024;  // slack to align the base to 1024
@@ -168,13 +166,10 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 
 // One work unit: query pair qp (rows qp*256 .. +255) of head bh, over the KV tiles
 // [kv0, kv0 + n[t]) for query tile t (0 tiles when the query tile lies past Sq or,
-// causally, before the range).  Units are numbered so that non-causal grids keep a
-// head's query pairs adjacent (concurrent units share its K/V in L2) and causal grids
-// take the heads in groups of p.head_group (the last group may be smaller), each
-// group's units heaviest first (the last query pairs of the group's heads first): the
-// units in flight then span about one group, whose K/V the host sized to fit in part
-// of L2, instead of every head.  The KV ranges of one (query pair, head) are
-// adjacent.
+// causally, before the range).  Units are numbered so that causal grids go heaviest
+// first (the last query pairs of every head first) and non-causal grids keep a head's
+// query pairs adjacent (concurrent units share its K/V in L2); the KV ranges of one
+// (query pair, head) are adjacent.
 struct Unit {
     int qp, bh, split, kv0;
     int n[2];
@@ -202,12 +197,8 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
     w.split = SPLIT ? u % p.n_splits : 0;
     const int rest = SPLIT ? u / p.n_splits : u;
     if constexpr (CAUSAL) {
-        const int per_group = p.head_group * p.n_qp;
-        const int g = rest / per_group;
-        const int within = rest - g * per_group;
-        const int hg = min(p.head_group, p.BH - g * p.head_group);
-        w.qp = p.n_qp - 1 - within / hg;
-        w.bh = g * p.head_group + within % hg;
+        w.qp = p.n_qp - 1 - rest / p.BH;
+        w.bh = rest % p.BH;
     } else {
         w.qp = rest % p.n_qp;
         w.bh = rest / p.n_qp;
@@ -258,42 +249,11 @@ __device__ __forceinline__ void scores_ready(uint32_t (&s)[128], int half) {
     }
 }
 
-#ifndef ATTN_EXP_POLY_PER8
-#define ATTN_EXP_POLY_PER8 0
-#endif
-
-// 2^x for a pair of values on the FMA pipe instead of the SFU: x = n + f with n =
-// round(x) (the magic-number addition: 1.5 * 2^23 + 127 puts n + 127 in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted here (weighted least
-// squares iterated to the equioscillating minimax, relative error 7.5e-5 on
-// [-1/2, 1/2], far below the 16-bit rounding of P); 2^n from the exponent field
-// (n + 127) << 23.  x is clamped to [-127, 127]: 2^-127 becomes exactly 0, and 2^127
-// still exceeds any row-sum limit.
-__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
-    constexpr float MAGIC = 12583039.0f;  // 1.5 * 2^23 + 127
-    x0 = fminf(fmaxf(x0, -127.f), 127.f);
-    x1 = fminf(fmaxf(x1, -127.f), 127.f);
-    const uint64_t x2 = ptx::f32x2(x0, x1);
-    const uint64_t mg = ptx::f32x2(MAGIC, MAGIC);
-    const uint64_t t2 = ptx::add2(x2, mg);
-    const uint64_t f2 = ptx::sub2(x2, ptx::sub2(t2, mg));
-    uint64_t q = ptx::fma2(f2, ptx::f32x2(0x1.c3f6a6p-5f, 0x1.c3f6a6p-5f),
-                           ptx::f32x2(0x1.f0ddccp-3f, 0x1.f0ddccp-3f));
-    q = ptx::fma2(q, f2, ptx::f32x2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
-    q = ptx::fma2(q, f2, ptx::f32x2(0x1.fff694p-1f, 0x1.fff694p-1f));
-    float t0, t1;
-    ptx::f32x2_split(t2, t0, t1);
-    return ptx::mul2(q, ptx::f32x2(__uint_as_float(__float_as_uint(t0) << 23),
-                                   __uint_as_float(__float_as_uint(t1) << 23)));
-}
-
 // p = 2^(s * c - m) for 32 column pairs starting at pair k0, packed to 16 bits into
-// pk; the row sum of the p as computed accumulates in the packed pair acc and, for
-// bf16, the row sum of the p as rounded (the weights P V actually applies) in accr.
+// pk, the row sum accumulated in the packed pair acc.
 template <bool IS_BF16>
 __device__ __forceinline__ void exp_pairs32(const uint32_t (&s)[128], int k0, float c,
-                                            float neg_m, uint32_t (&pk)[64], uint64_t& acc,
-                                            uint64_t& accr) {
+                                            float neg_m, uint32_t (&pk)[64], uint64_t& acc) {
     const uint64_t c2 = ptx::f32x2(c, c), m2 = ptx::f32x2(neg_m, neg_m);
 #pragma unroll
     for (int k = k0; k < k0 + 32; ++k) {
@@ -301,41 +261,16 @@ __device__ __forceinline__ void exp_pairs32(const uint32_t (&s)[128], int k0, fl
         ptx::f32x2_split(
             ptx::fma2(ptx::f32x2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2, m2),
             x0, x1);
-        float p0, p1;
-        if ((k & 7) < ATTN_EXP_POLY_PER8) {
-            ptx::f32x2_split(exp2_poly_pair(x0, x1), p0, p1);
-        } else {
-            p0 = ptx::ex2(x0);
-            p1 = ptx::ex2(x1);
-        }
+        const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
         acc = ptx::add2(acc, ptx::f32x2(p0, p1));
         pk[k] = pack2<IS_BF16>(p0, p1);
-        if constexpr (IS_BF16)  // a bf16 value is the upper half of its fp32 pattern
-            accr = ptx::add2(accr, ptx::f32x2(__uint_as_float(pk[k] << 16),
-                                              __uint_as_float(pk[k] & 0xffff0000u)));
     }
 }
 
-// Row normalisers: l, the sum of the p as computed in fp32 (for the log-sum-exp), and
-// lr, the sum of the p as rounded to 16 bits for P V (O is divided by it, so O is an
-// exact convex combination of the V rows under the weights P V applied: a near one-hot
-// row then loses nothing to the rounding of its dominant p).  fp16 rounds P four times
-// finer than bf16 and keeps lr = l.
-struct RowSums {
-    float l, lr;
-};
-
-template <bool IS_BF16>
-__device__ __forceinline__ void add_sums(RowSums& r, float alpha, uint64_t acc, uint64_t accr) {
+__device__ __forceinline__ float sum_pair(uint64_t acc) {
     float a0, a1;
     ptx::f32x2_split(acc, a0, a1);
-    r.l = r.l * alpha + (a0 + a1);
-    if constexpr (IS_BF16) {
-        ptx::f32x2_split(accr, a0, a1);
-        r.lr = r.lr * alpha + (a0 + a1);
-    } else {
-        r.lr = r.l;
-    }
+    return a0 + a1;
 }
 
 // One KV tile of the query row this thread owns, with the masking decided at compile
@@ -349,7 +284,7 @@ __device__ __forceinline__ void add_sums(RowSums& r, float alpha, uint64_t acc, 
 // scaled by before P_j V_j is added (1 = none).
 template <bool IS_BF16, bool NEG, bool MASK, bool GEN>
 __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, float c,
-                                                   float& m_used, RowSums& l) {
+                                                   float& m_used, float& l) {
     uint32_t s[128];
     load_scores<NEG>(tS, s, 0);
     ptx::tmem_wait_ld();
@@ -390,51 +325,49 @@ __device__ __forceinline__ float softmax_tile_body(uint32_t tS, int j, int lim, 
     // p = 2^(s * c - m): scale and shift in one packed fma per column pair; the row
     // sums accumulate in packed pairs too (masked scores are -inf and c > 0, so their p
     // is exactly 0)
-    uint64_t acc = ptx::f32x2(0.f, 0.f), accr = acc;
+    uint64_t acc = ptx::f32x2(0.f, 0.f);
     uint32_t pk[64];
-    exp_pairs32<IS_BF16>(s, 0, c, neg_m, pk, acc, accr);
-    exp_pairs32<IS_BF16>(s, 32, c, neg_m, pk, acc, accr);
-    add_sums<IS_BF16>(l, alpha, acc, accr);
+    exp_pairs32<IS_BF16>(s, 0, c, neg_m, pk, acc);
+    exp_pairs32<IS_BF16>(s, 32, c, neg_m, pk, acc);
+    l = l * alpha + sum_pair(acc);
     ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
     ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
     return alpha;
 }
 
 
-// A row sum of one tile's p above this means some p exceeded 2^8 (the lazy threshold:
-// 128 values of at most 2^8 sum to at most 2^15), i.e. the row's maximum moved up by
-// more than the threshold: the tile is redone with the new maximum.  Every p that is
-// kept is at most 2^15, inside the fp16 range.
-constexpr float RUNNING_SUM_LIMIT = 32768.0f;
-
-// An unmasked KV tile after the first of a row's range, without a row-max pass: the
-// running max the row already has (m_used, finite) is used directly, p = 2^(s c -
-// m_used), and the row max of the tile is only needed when the tile's row sum shows
-// that it moved up by more than the lazy threshold.  A warp with such a row (rare:
-// the running max settles within the first tiles) reloads its scores from tensor
-// memory, takes the row max as the first tile does, and recomputes; rows of the warp
-// whose max did not move recompute the same values.  The result equals the row-max
-// path's: the kept max never trails the true one by more than the threshold, and O
-// and l are relative to the same kept max.  Returns alpha as softmax_tile_body does.
-template <bool IS_BF16, bool NEG>
+// An unmasked KV tile after the first of a row's range, without a row-max pass in the
+// common case: the running max the row already has (m_used, finite) is used directly,
+// p = 2^(s c - m_used), and the tile's row max is only taken when the row sum exceeds
+// 2^LIMIT_LOG2, which every tile whose max stays within LIMIT_LOG2 - 7 of the kept
+// one passes (128 values of at most 2^(LIMIT_LOG2 - 7)).  A warp with a row above the
+// limit (rare once the first tiles have set the max) reloads its scores from tensor
+// memory (P is not written yet), takes the row max, moves the kept max to it when it
+// is higher (so the dominant p is then exactly 1) and recomputes; rows of the warp
+// whose max did not move recompute the same values.  O and l stay relative to the same
+// kept max, so O / l is unchanged, and every kept p is at most 2^LIMIT_LOG2.
+// LIMIT_LOG2 = 15 keeps every p inside fp16; 8 matches the lazy threshold of the
+// row-max path, so a jump in the max by more than 2^8 always leaves the dominant p
+// exactly 1 (one-hot rows then lose nothing to the rounding of their dominant p).
+// Returns alpha, as softmax_tile_body does.
+template <bool IS_BF16, bool NEG, int LIMIT_LOG2>
 __device__ __forceinline__ float softmax_tile_running(uint32_t tS, float c, float& m_used,
-                                                      RowSums& l) {
+                                                      float& l) {
+    constexpr float LIMIT = static_cast<float>(1 << LIMIT_LOG2);
     uint32_t s[128];
     uint32_t pk[64];
-    uint64_t acc = ptx::f32x2(0.f, 0.f), accr = acc;
+    uint64_t acc = ptx::f32x2(0.f, 0.f);
     load_scores<NEG>(tS, s, 0);
     ptx::tmem_wait_ld();
     scores_ready<NEG>(s, 0);
     // the second half's load runs under the first half's exponentials
     load_scores<NEG>(tS, s, 1);
-    exp_pairs32<IS_BF16>(s, 0, c, -m_used, pk, acc, accr);
+    exp_pairs32<IS_BF16>(s, 0, c, -m_used, pk, acc);
     ptx::tmem_wait_ld();
     scores_ready<NEG>(s, 1);
-    exp_pairs32<IS_BF16>(s, 32, c, -m_used, pk, acc, accr);
-    float sum0, sum1;
-    ptx::f32x2_split(acc, sum0, sum1);
+    exp_pairs32<IS_BF16>(s, 32, c, -m_used, pk, acc);
     float alpha = 1.f;
-    if (__any_sync(0xffffffffu, sum0 + sum1 > RUNNING_SUM_LIMIT)) {
+    if (__any_sync(0xffffffffu, sum_pair(acc) > LIMIT)) {
         load_scores<NEG>(tS, s, 0);
         load_scores<NEG>(tS, s, 1);
         ptx::tmem_wait_ld();
@@ -448,36 +381,32 @@ __device__ __forceinline__ float softmax_tile_running(uint32_t tS, float c, floa
         const float mx = ptx::max3(ptx::max3(a[0], a[1], a[2]), ptx::max3(a[3], a[4], a[5]),
                                    fmaxf(a[6], a[7]));
         const float m_tile = mx * c;
-        if (m_tile > m_used + LAZY_RESCALE_LOG2) {
+        if (m_tile > m_used) {
             alpha = ptx::ex2(m_used - m_tile);
             m_used = m_tile;
         }
-        acc = accr = ptx::f32x2(0.f, 0.f);
-        exp_pairs32<IS_BF16>(s, 0, c, -m_used, pk, acc, accr);
-        exp_pairs32<IS_BF16>(s, 32, c, -m_used, pk, acc, accr);
+        acc = ptx::f32x2(0.f, 0.f);
+        exp_pairs32<IS_BF16>(s, 0, c, -m_used, pk, acc);
+        exp_pairs32<IS_BF16>(s, 32, c, -m_used, pk, acc);
     }
-    add_sums<IS_BF16>(l, alpha, acc, accr);
+    l = l * alpha + sum_pair(acc);
     ptx::tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
     ptx::tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
     return alpha;
 }
 
-// The tile's masking is decided once, by a warp-uniform branch, so the unmasked tiles
-// (all but the last and, causally, the diagonal ones) run the loops without it; with
-// RUNNING an unmasked tile after the first of the range also skips the row-max pass.
-// row_vis: the last key this row sees; tile_vis_min: the least of that over the
-// tile's rows (causal only).
-template <bool IS_BF16, bool CAUSAL, bool NEG, bool GEN, bool RUNNING = true>
+// LIMIT_LOG2: see softmax_tile_running.
+template <bool IS_BF16, bool CAUSAL, bool NEG, bool GEN, int LIMIT_LOG2>
 __device__ __forceinline__ float softmax_tile(uint32_t tS, int j, int kv0, int Sk, int row_vis,
                                               int tile_vis_min, float c, float& m_used,
-                                              RowSums& l) {
+                                              float& l) {
     const bool need_mask = (kv0 + BN > Sk) || (CAUSAL && kv0 + BN - 1 > tile_vis_min);
     if (need_mask) {
         int lim = Sk - 1 - kv0;
         if (CAUSAL) lim = min(lim, row_vis - kv0);
         return softmax_tile_body<IS_BF16, NEG, true, GEN>(tS, j, lim, c, m_used, l);
     }
-    if (RUNNING && j > 0) return softmax_tile_running<IS_BF16, NEG>(tS, c, m_used, l);
+    if (j > 0) return softmax_tile_running<IS_BF16, NEG, LIMIT_LOG2>(tS, c, m_used, l);
     return softmax_tile_body<IS_BF16, NEG, false, GEN>(tS, j, 0, c, m_used, l);
 }
 
@@ -554,7 +483,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t sV = sbase + L::V_OFF;
     float* s_fm = reinterpret_cast<float*>(smem + L::FM_OFF);
     float* s_fl = reinterpret_cast<float*>(smem + L::FL_OFF);
-    float* s_fr = reinterpret_cast<float*>(smem + L::FR_OFF);
     const uint32_t bars = sbase + L::BAR_OFF;
     auto B_QF = [&](int t) { return bars + 8u * t; };                  // Q_t loaded
     auto B_KF = [&](int s) { return bars + 8u * (2 + s); };
@@ -566,8 +494,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto B_OF = [&](int t) { return bars + 8u * (6 + 4 * NS + t); };   // last PV_t done
     auto B_ST = [&](int t) { return bars + 8u * (8 + 4 * NS + t); };   // final m, l in smem
     auto B_OE = [&](int t) { return bars + 8u * (10 + 4 * NS + t); };  // O_t, m, l read out
-    const uint32_t B_QE = bars + 8u * (12 + 4 * NS);                   // Q tiles free
-    const uint32_t B_DR = bars + 8u * (13 + 4 * NS);
+    auto B_QE = [&](int t) { return bars + 8u * (12 + 4 * NS + t); };  // Q_t free
+    const uint32_t B_DR = bars + 8u * (14 + 4 * NS);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     Ctx ctx{reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4)};
     const int n_units = p.n_qp * p.BH * p.n_splits;
@@ -588,7 +516,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_init(B_VF(s), 1);
             ptx::mbar_init(B_VE(s), 1);
         }
-        ptx::mbar_init(B_QE, 1);
+        ptx::mbar_init(B_QE(0), 1);
+        ptx::mbar_init(B_QE(1), 1);
         ptx::mbar_init(B_DR, 1);
         *ctx.err = 0;
         ptx::fence_mbar_init();
@@ -639,12 +568,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tile_vis_min = tile_vis<true>(q0t, min(q0t + BM - 1, p.Sq - 1), p);
             }
             float m_used = -INFINITY;
-            RowSums l{0.f, 0.f};
+            float l = 0.f;
             for (int j = 0; j < n_t; ++j, ++it) {
                 if (!(ok = warp_wait(ctx, B_SF(t), it & 1))) break;
                 ptx::tc_fence_after();
                 const int kt = DEC ? 2 * j + t : j;  // the KV tile within the unit's range
-                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG, GEN>(
+                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG, GEN, 15>(
                     tS, j, (w.kv0 + kt) * BN, p.Sk, row_vis, tile_vis_min, c_abs, m_used, l);
                 // O_t holds the sum over tiles < j (PV_t,j-1 completed before S_t,j);
                 // bring it to the new max before PV_t,j adds to it
@@ -670,8 +599,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // the epilogue must be done with the previous unit's statistics
             if (!(ok = warp_wait(ctx, B_OE(t), (ut & 1) ^ 1))) break;
             s_fm[t * BM + row] = m_used;
-            s_fl[t * BM + row] = l.l;
-            s_fr[t * BM + row] = l.lr;
+            s_fl[t * BM + row] = l;
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(B_ST(t));
             ++ut;
@@ -705,18 +633,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (!(ok = warp_wait(ctx, B_OF(1), ut[1] & 1))) break;
                 }
                 ptx::tc_fence_after();
-                const float m0 = s_fm[row], l0 = s_fl[row], r0 = s_fr[row];
+                const float m0 = s_fm[row], l0 = s_fl[row];
                 const float m1 = nt1 > 0 ? s_fm[BM + row] : -INFINITY;
                 const float l1 = nt1 > 0 ? s_fl[BM + row] : 0.f;
-                const float r1 = nt1 > 0 ? s_fr[BM + row] : 0.f;
                 const float mx = fmaxf(m0, m1);
-                // weights of the halves (0 for a half that saw no key); O is divided by
-                // the rounded sums, the LSE takes the computed ones
+                // weights of the halves (0 for a half that saw no key)
                 const float a0 = m0 == -INFINITY ? 0.f : ptx::ex2(m0 - mx);
                 const float a1 = m1 == -INFINITY ? 0.f : ptx::ex2(m1 - mx);
                 const float lt = l0 * a0 + l1 * a1;
-                const float rt = r0 * a0 + r1 * a1;
-                const float inv = rt > 0.f ? 1.f / rt : 0.f;
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
                 const float w0 = a0 * inv, w1 = a1 * inv;
                 const float lse_row =
                     lt > 0.f ? (mx + log2f(lt)) * 0.69314718055994530942f : -INFINITY;
@@ -766,10 +691,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 ptx::tc_fence_after();
                 const float m_used = s_fm[t * BM + row];
                 const float l = s_fl[t * BM + row];
-                const float lr = s_fr[t * BM + row];
-                // l = 0 only for a row with no visible key in a split range; O is divided
-                // by the sum of the rounded p, the LSE takes the computed sum
-                const float inv_l = lr > 0.f ? 1.f / lr : 0.f;
+                // l = 0 only for a row with no visible key in a split range
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
                 const float lse_row =
                     l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
                 const uint32_t tO = tmem + lane_base + TMEM_O + D * t;
@@ -900,7 +823,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ptx::tc_fence_after();
                         issue_s(j, slot(j));
                         ptx::mma_commit(B_KE(slot(j)));
-                        if (j == n - 1) ptx::mma_commit(B_QE);  // the unit's last S is issued
+                        if (j == n - 1) ptx::mma_commit(B_QE(0));  // the unit's last S is issued
                     }
                     for (int j = 0; ok && j < n; ++j) {
                         const int t = j & 1, i = j >> 1;
@@ -919,13 +842,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             ptx::tc_fence_after();
                             issue_s(t, slot(j + 2));
                             ptx::mma_commit(B_KE(slot(j + 2)));
-                            if (j + 2 == n - 1) ptx::mma_commit(B_QE);  // last S issued
+                            if (j + 2 == n - 1) ptx::mma_commit(B_QE(0));  // last S issued
                         }
                     }
                     for (int t = 0; t < 2; ++t) ut[t] += nt[t] > 0 ? 1u : 0u;
                     kv += static_cast<uint32_t>(n);
                     ++nu;
                 }
+                // Tile 0 runs ahead across units: once its last P V of a unit is issued,
+                // the next unit's S_0,0 follows at once (its Q_0 and K_0 loaded: tested
+                // without blocking, else after tile 1's work of that step), so the two
+                // tiles' softmaxes stay half a period apart across the unit boundary and,
+                // causally, tile 0 works while tile 1 finishes its extra diagonal tile.
+                // Deadlock-free: the producer loads Q_0, K_0, Q_1, V_0, K_1, ... of a
+                // unit; Q_0 of the next unit needs only tile 0's last S of this unit
+                // (Q_t is freed per tile), and K_0 of the next unit needs the ring slot
+                // of K at tile n_max - NS of this unit, whose S MMAs were issued before
+                // tile 0's last step when n_0 >= n_max - NS + 1 (the lookahead's
+                // condition).
+                bool s0_pre = false;  // S_0,0 of the unit about to start is issued
+                auto next_unit = [&](int r0, Unit& nx) {
+                    for (int r1 = r0 + 1;; ++r1) {
+                        const int u1 = unit_of(r1, n_units);
+                        if (u1 < 0) return false;
+                        nx = decode_unit<CAUSAL, SPLIT, GEN>(u1, p);
+                        if (max(nx.n[0], nx.n[1]) > 0) return true;
+                    }
+                };
                 for (int r = 0; !DEC && ok; ++r) {
                     const int u = unit_of(r, n_units);
                     if (u < 0) break;
@@ -935,15 +878,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     if (n_max == 0) continue;  // a split range no query row of the unit sees
                     auto slot = [&](int j) { return static_cast<int>((kv + j) % NS); };
                     auto phase = [&](int j) { return ((kv + j) / NS) & 1u; };
-                    if (!(ok = wait_bounded(ctx, B_QF(0), nu & 1) &&
+                    if (!(ok = (s0_pre || wait_bounded(ctx, B_QF(0), nu & 1)) &&
                                wait_bounded(ctx, B_QF(1), nu & 1) &&
                                wait_bounded(ctx, B_KF(slot(0)), phase(0))))
                         break;
                     ptx::tc_fence_after();
-                    for (int t = 0; t < 2; ++t)
-                        if (n_t[t] > 0) issue_s(t, slot(0));
+                    if (n_t[0] > 0 && !s0_pre) issue_s(0, slot(0));
+                    if (n_t[1] > 0) issue_s(1, slot(0));
                     ptx::mma_commit(B_KE(slot(0)));
-                    if (n_max == 1) ptx::mma_commit(B_QE);  // the unit's last S is issued
+                    // Q_t is free once the unit's last S_t is issued (or it has none)
+                    if (n_t[0] <= 1 && !s0_pre) ptx::mma_commit(B_QE(0));
+                    if (n_t[1] <= 1) ptx::mma_commit(B_QE(1));
+                    s0_pre = false;
+                    Unit nx;
+                    const bool ahead = n_t[0] > 0 && n_t[0] >= n_max - NS + 1 &&
+                                       next_unit(r, nx) && nx.n[0] > 0;
+                    bool pending = false;  // the lookahead waits for its Q_0 / K_0
+                    auto issue_ahead = [&]() {
+                        ptx::tc_fence_after();
+                        issue_s(0, slot(n_max));
+                        if (nx.n[0] == 1) ptx::mma_commit(B_QE(0));
+                        s0_pre = true;
+                    };
                     for (int j = 0; ok && j < n_max; ++j) {
                         const bool nxt = j + 1 < n_max;
                         if (nxt && !(ok = wait_bounded(ctx, B_KF(slot(j + 1)), phase(j + 1))))
@@ -960,14 +916,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             ptx::tc_fence_after();
                             issue_pv(t, slot(j), j == 0);
                             if (j == n_t[t] - 1) ptx::mma_commit(B_OF(t));
-                            if (j + 1 < n_t[t]) issue_s(t, slot(j + 1));
+                            if (j + 1 < n_t[t]) {
+                                issue_s(t, slot(j + 1));
+                                if (j + 1 == n_t[t] - 1) ptx::mma_commit(B_QE(t));
+                            } else if (t == 0 && ahead) {
+                                if (ptx::mbar_test_wait(B_QF(0), (nu + 1) & 1) &&
+                                    ptx::mbar_test_wait(B_KF(slot(n_max)), phase(n_max)))
+                                    issue_ahead();
+                                else
+                                    pending = true;
+                            }
                         }
                         if (!ok) break;
-                        ptx::mma_commit(B_VE(slot(j)));
-                        if (nxt) {
-                            ptx::mma_commit(B_KE(slot(j + 1)));
-                            if (j + 1 == n_max - 1) ptx::mma_commit(B_QE);  // last S issued
+                        if (pending) {
+                            if (!(ok = wait_bounded(ctx, B_QF(0), (nu + 1) & 1) &&
+                                       wait_bounded(ctx, B_KF(slot(n_max)), phase(n_max))))
+                                break;
+                            issue_ahead();
+                            pending = false;
                         }
+                        ptx::mma_commit(B_VE(slot(j)));
+                        if (nxt) ptx::mma_commit(B_KE(slot(j + 1)));
                     }
                     for (int t = 0; t < 2; ++t) ut[t] += n_t[t] > 0 ? 1u : 0u;
                     kv += static_cast<uint32_t>(n_max);
@@ -984,7 +953,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const bool load_q = !(p.flags & FLAG_SKIP_Q_LOAD);
                 uint32_t kv = 0, nu = 0;
                 int64_t last_k = -1, last_v = -1;  // ring positions of the last K / V issued
-                int64_t last_q = -1;               // unit count at the last Q load
+                int64_t last_q[2] = {-1, -1};      // unit count at the last Q_t load
                 bool ok = true;
                 for (int r = 0; ok; ++r) {
                     const int u = unit_of(r, n_units);
@@ -994,18 +963,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int bh = w.bh;
                     const int n_max = max(w.n[0], w.n[1]);
                     if (n_max == 0) continue;  // nothing to load (the MMA skips it too)
-                    // Q_0, Q_1 are free once the previous unit's S MMAs completed
-                    // (DEC: only Q_0 is used)
-                    if (!(ok = wait_bounded(ctx, B_QE, (nu & 1) ^ 1))) break;
-                    if (load_q) {
-                        for (int t = 0; t < (DEC ? 1 : 2); ++t) {
-                            ptx::mbar_arrive_expect_tx(B_QF(t), L::TILE_BYTES);
-                            for (int c = 0; c < L::NCH; ++c)
-                                ptx::tma_load_3d(sQ + t * L::TILE_BYTES + c * CHUNK_BYTES, &tm_q,
-                                                 B_QF(t), c * CHUNK_ELEMS, q0 + BM * t, bh);
-                        }
-                        last_q = nu;
-                    }
+                    // Q_t is free once the previous unit's S_t MMAs completed.  Order of
+                    // the loads: Q_0, K_0, Q_1, V_0, K_1, V_1, ... (DEC: only Q_0 is used)
+                    auto load_q_tile = [&](int t) {
+                        if (!(ok = wait_bounded(ctx, B_QE(t), (nu & 1) ^ 1))) return;
+                        if (!load_q) return;
+                        ptx::mbar_arrive_expect_tx(B_QF(t), L::TILE_BYTES);
+                        for (int c = 0; c < L::NCH; ++c)
+                            ptx::tma_load_3d(sQ + t * L::TILE_BYTES + c * CHUNK_BYTES, &tm_q,
+                                             B_QF(t), c * CHUNK_ELEMS, q0 + BM * t, bh);
+                        last_q[t] = nu;
+                    };
+                    load_q_tile(0);
                     for (int j = 0; ok && j < n_max; ++j) {
                         const uint32_t pos = kv + j;
                         const int s = static_cast<int>(pos % NS);
@@ -1016,6 +985,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             ptx::tma_load_3d(sK + s * L::TILE_BYTES + c * CHUNK_BYTES, &tm_k,
                                              B_KF(s), c * CHUNK_ELEMS, (w.kv0 + j) * BN, bh);
                         last_k = pos;
+                        if (!DEC && j == 0) {
+                            load_q_tile(1);
+                            if (!ok) break;
+                        }
                         if (!(ok = wait_bounded(ctx, B_VE(s), ph ^ 1))) break;
                         ptx::mbar_arrive_expect_tx(B_VF(s), L::TILE_BYTES);
                         for (int c = 0; c < L::NCH; ++c)
@@ -1027,10 +1000,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     ++nu;
                 }
                 // Let every copy this thread started land before the CTA can exit.
-                if (last_q >= 0) {
-                    wait_drain(B_QF(0), static_cast<uint32_t>(last_q) & 1);
-                    if (!DEC) wait_drain(B_QF(1), static_cast<uint32_t>(last_q) & 1);
-                }
+                for (int t = 0; t < 2; ++t)
+                    if (last_q[t] >= 0) wait_drain(B_QF(t), static_cast<uint32_t>(last_q[t]) & 1);
                 for (int64_t q = (last_k - NS + 1 > 0 ? last_k - NS + 1 : 0); q <= last_k; ++q)
                     wait_drain(B_KF(static_cast<int>(q % NS)), (q / NS) & 1);
                 for (int64_t q = (last_v - NS + 1 > 0 ? last_v - NS + 1 : 0); q <= last_v; ++q)

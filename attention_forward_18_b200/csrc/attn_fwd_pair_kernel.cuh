@@ -68,8 +68,7 @@ struct Layout {
     static constexpr int V_OFF = K_OFF + NSK * K_BYTES;
     static constexpr int FM_OFF = V_OFF + NSV * V_BYTES;  // final max float [128]
     static constexpr int FL_OFF = FM_OFF + BM * 4;       // final sum float [128]
-    static constexpr int FR_OFF = FL_OFF + BM * 4;       // final rounded sum float [128]
-    static constexpr int BAR_OFF = FR_OFF + BM * 4;
+    static constexpr int BAR_OFF = FL_OFF + BM * 4;
     // q_full, q_empty, k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV], then at
     // BASE: s_full[2], p_full[2], pv_done, o_final, stats, o_free, drain
     static constexpr int BASE = 2 + 2 * NSK + 2 * NSV;
@@ -129,7 +128,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t sV = sbase + L::V_OFF;
     float* s_fm = reinterpret_cast<float*>(smem + L::FM_OFF);
     float* s_fl = reinterpret_cast<float*>(smem + L::FL_OFF);
-    float* s_fr = reinterpret_cast<float*>(smem + L::FR_OFF);
     const uint32_t bars = sbase + L::BAR_OFF;
     const uint32_t B_QF = bars, B_QE = bars + 8u;
     auto B_KF = [&](int s) { return bars + 8u * (2 + s); };
@@ -215,7 +213,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tile_vis_min = tile_vis<true>(q0t, min(q0t + BM - 1, p.Sq - 1), p);
             }
             float m_used = -INFINITY;
-            RowSums l{0.f, 0.f};
+            float l = 0.f;
             for (int j = 0; j < n; ++j, ++gt) {
                 const int b = j & 1;
                 if (!(ok = warp_wait_cl(ctx, B_SF(b), sfc[b] & 1))) break;
@@ -227,7 +225,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 ptx::tc_fence_after();
                 // (the pair runs the larger KV range of its two query tiles, so causal rows
                 // can meet tiles, even a first tile, with no visible key: keep the guard)
-                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG, CAUSAL>(
+                // (a row-sum limit of 2^8: a jump in a row's max by more than the lazy
+                // threshold always leaves its dominant p exactly 1)
+                const float alpha = softmax_tile<IS_BF16, CAUSAL, NEG, CAUSAL, 8>(
                     tmem + lane_base + 128u * b, j, (w.kv0 + j) * BN, p.Sk, row_vis,
                     tile_vis_min, c_abs, m_used, l);
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -256,8 +256,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (!ok) continue;
             if (!(ok = warp_wait_cl(ctx, B_OE, (ut & 1) ^ 1))) break;
             s_fm[row] = m_used;
-            s_fl[row] = l.l;
-            s_fr[row] = l.lr;
+            s_fl[row] = l;
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(B_ST);
             ++ut;
@@ -287,9 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_fence_after();
             const float m_used = s_fm[row];
             const float l = s_fl[row];
-            // O divided by the sum of the rounded p, the LSE from the computed sum
-            const float lr = s_fr[row];
-            const float inv_l = lr > 0.f ? 1.f / lr : 0.f;
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
             const float lse_row =
                 l > 0.f ? (m_used + log2f(l)) * 0.69314718055994530942f : -INFINITY;
             const uint32_t tO = tmem + lane_base + TMEM_O;

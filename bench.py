@@ -563,7 +563,7 @@ def decode_workloads(names):
         lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
         dcode = af.ATTN_F16 if w.dtype == "f16" else af.ATTN_BF16
         Hkv = w.kv_heads
-        n = af.ex_default_splits(w.B, w.H, Hkv, w.Sq, w.Sk, af.ATTN_MASK_NONE)
+        n = af.ex_default_splits(w.B, w.H, Hkv, w.Sq, w.Sk, af.ATTN_MASK_NONE, w.D)
         nbytes = af.splitkv_workspace_bytes(w.B, w.H, w.Sq, w.D, n)
         ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
@@ -869,7 +869,7 @@ def profile_extra(spec):
         if cut:
             w = dataclasses.replace(w, B=int(cut))
         q, k, v = (t.cuda() for t in make_inputs(w))
-        n = af.ex_default_splits(w.B, w.H, w.kv_heads, w.Sq, w.Sk, af.ATTN_MASK_NONE)
+        n = af.ex_default_splits(w.B, w.H, w.kv_heads, w.Sq, w.Sk, af.ATTN_MASK_NONE, w.D)
         af.attention_ex(q, k, v, mask=af.ATTN_MASK_NONE, scale=w.scale, n_splits=n)
         shape = f"B={w.B} H={w.H} Hkv={w.kv_heads} Sq={w.Sq} Sk={w.Sk} D={w.D} splits={n}"
     elif name in SOFTMAX_WORKLOADS:

@@ -116,9 +116,10 @@ int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
  * of the full normaliser; a range no key of which a row sees has LSE_s = -inf).  The
  * pages describe the online-softmax rescaling this relies on; the split itself is this
  * library's (no counterpart on the pages).
- *   n_splits   1 .. 1024 ranges of ceil(ceil(Sk/128) / n_splits) 128-key tiles each
- *              (trailing ranges may be empty); attn_fwd_splitkv_default_splits picks
- *              one for the device
+ *   n_splits   1 .. 1024 ranges of ceil(ceil(Sk/T) / n_splits) T-key tiles each, T = 128
+ *              (T = 64 for D = 192 / 256 with at most 128 query rows, the decode shapes
+ *              of the wide kernel); trailing ranges may be empty;
+ *              attn_fwd_splitkv_default_splits picks one for the device
  *   workspace  device, 256-byte aligned, at least attn_fwd_splitkv_workspace_bytes(B,
  *              H, Sq, D, n_splits) bytes, caller-owned, not overlapping any argument;
  *              its contents are scratch (overwritten each call)
@@ -151,14 +152,16 @@ int attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse
                 attn_stream_t stream);
 
 /* attn_fwd_splitkv_default_splits for attn_fwd_ex's arguments (0 for invalid ones). */
-int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int mask);
+int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int D, int mask);
 
 /* Bytes of workspace attn_fwd_splitkv needs (0 for invalid arguments). */
 size_t attn_fwd_splitkv_workspace_bytes(int B, int H, int Sq, int D, int n_splits);
 
 /* A split count for these sizes on the current device: the one that balances
- * (query block, head, range) units over the SMs best (1 .. 1024; 0 for invalid sizes). */
-int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int causal);
+ * (query block, head, range) units over the SMs best, counted in the geometry of the
+ * kernel that runs D (its query rows and keys per tile, and two SMs per unit on the
+ * D = 192 / 256 CTA pairs) (1 .. 1024; 0 for invalid sizes). */
+int attn_fwd_splitkv_default_splits(int B, int H, int Sq, int Sk, int D, int causal);
 
 /* Size of the scratch attn_fwd_splitkv_noalloc uses in place of a workspace. */
 #define ATTN_SPLITKV_NOALLOC_SCRATCH_BYTES (16u << 20)
@@ -203,7 +206,7 @@ int attn_fwd_status(attn_stream_t stream, int *device_status);
 /* Static string naming an ATTN_* code (never NULL). */
 const char *attn_fwd_strerror(int code);
 
-/* ABI version of this header, currently 1. */
+/* ABI version of this header, currently 2 (the split-count helpers take D). */
 int attn_fwd_abi_version(void);
 
 /*

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_strerror():
-    assert af.abi_version() == 1
+    assert af.abi_version() == 2
     for code in range(0, -14, -1):
         msg = af.strerror(code)
         assert msg and msg != "unknown error code", code
@@ -152,6 +152,22 @@ def test_splitkv_default_splits_in_range():
     assert af.splitkv_default_splits(1, 8, 1, 131072, causal=True) == 1
     # many units already fill the SMs
     assert af.splitkv_default_splits(64, 32, 256, 256) == 1
+
+
+def test_default_splits_follow_the_kernel_geometry_of_D():
+    # no device here: the library assumes 148 SMs.  4 single-row heads, 16384 keys: the
+    # D = 128 kernel's 128 tiles of 128 keys fill 128 SMs best with 32 ranges; the wide
+    # kernel's 256 tiles of 64 keys (D = 256 decode shapes) with 37 ranges of 7 tiles
+    assert af.splitkv_default_splits(1, 4, 1, 16384, D=128) == 32
+    assert af.splitkv_default_splits(1, 4, 1, 16384, D=256) == 37
+    # 300 query rows at D = 256 run on CTA pairs (two SMs a unit): 4 units over 74 pairs
+    # take 18 ranges, where 148 single-SM units would take 37
+    assert af.splitkv_default_splits(1, 2, 300, 65536, D=128) == 37
+    assert af.splitkv_default_splits(1, 2, 300, 65536, D=256) == 18
+    assert af.ex_default_splits(1, 2, 2, 300, 65536, af.ATTN_MASK_NONE, D=192) == 18
+    # head dimensions outside the library's set
+    assert af.splitkv_default_splits(1, 4, 1, 16384, D=48) == 0
+    assert af.ex_default_splits(1, 4, 4, 1, 16384, af.ATTN_MASK_NONE, D=512) == 0
 
 
 @pytest.mark.parametrize("kw,code", [

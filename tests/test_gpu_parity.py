@@ -86,6 +86,16 @@ def test_unusual_scales(scale):
     check_full(1, 2, 130, 260, 128, "f16", False, seed=6, scale=scale)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_near_one_hot_rows_in_bf16(causal):
+    """Scale 0.5 at D = 128 in bf16: scores spread over tens of log2 units, the row max
+    jumps by more than the lazy threshold on later tiles, and |O| reaches max |v|
+    (about 4.5), where bf16's own rounding of O is 1/64: the error budget left for the
+    rounding of P is small."""
+    rep = check_full(2, 4, 300, 1500, 128, "bf16", causal, seed=19 + causal, scale=0.5)
+    record(f"near one-hot D128 bf16 causal={causal}", rep)
+
+
 def test_deterministic_and_stream():
     """Bitwise-identical results over repeated runs, also on a non-default stream."""
     q, k, v = (t.cuda() for t in make_qkv(2, 4, 700, 900, 128, "bf16", 12))

@@ -125,7 +125,7 @@ def test_decode_workloads_in_bench_configuration(name):
     from workloads import DECODE_WORKLOADS, make_inputs, sample_rows
     w = DECODE_WORKLOADS[name]
     q, k, v = make_inputs(w)
-    n = af.ex_default_splits(w.B, w.H, w.kv_heads, w.Sq, w.Sk, af.ATTN_MASK_NONE)
+    n = af.ex_default_splits(w.B, w.H, w.kv_heads, w.Sq, w.Sk, af.ATTN_MASK_NONE, w.D)
     dq, dk, dv = (t.cuda() for t in (q, k, v))
     o, lse = af.attention_ex(dq, dk, dv, mask=af.ATTN_MASK_NONE, scale=w.scale, n_splits=n)
     torch.cuda.synchronize()
