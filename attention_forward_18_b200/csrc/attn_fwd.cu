@@ -530,9 +530,10 @@ int mask_of(int causal) { return causal ? ATTN_MASK_CAUSAL : ATTN_MASK_NONE; }
 // Split count for `units` (query block, head) pairs over KV tiles 0..n_kv-1 on `slots`
 // units that run at once (SMs, or CTA pairs): persistent CTAs take units round-robin,
 // so a pass lasts about
-//   ceil(units * n / slots) rounds x (tiles per range + a fill of ~2 tiles);
+//   ceil(units * n / slots) rounds x (tiles per range + a fill of `fill` tiles)
+// (the fill of a range, ~2 tiles of 128 keys, is ~4 of the wide kernel's 64-key tiles);
 // the n with the least of that (the fewest splits among equals: less to merge).
-int balanced_splits(int64_t units, int n_kv, int slots) {
+int balanced_splits(int64_t units, int n_kv, int slots, int fill) {
     const int num_sms = slots;
     int best = 1;
     int64_t best_cost = INT64_MAX;
@@ -541,7 +542,7 @@ int balanced_splits(int64_t units, int n_kv, int slots) {
         const int chunk = (n_kv + n - 1) / n;
         if ((n_kv + chunk - 1) / chunk != n) continue;  // some range would be empty
         const int64_t rounds = (units * n + num_sms - 1) / num_sms;
-        const int64_t cost = rounds * (chunk + 2);
+        const int64_t cost = rounds * (chunk + fill);
         if (cost < best_cost) {
             best_cost = cost;
             best = n;
@@ -628,7 +629,8 @@ int attn_fwd_ex_default_splits(int B, int H, int H_kv, int Sq, int Sk, int D, in
     const int64_t units = (rows + q_units - 1) / q_units * B * H_kv;
     // with the top-left causal mask no row sees a key past min(Sq, Sk)
     const int keys = mask == ATTN_MASK_CAUSAL ? (Sq < Sk ? Sq : Sk) : Sk;
-    return balanced_splits(units, (keys + kv_keys - 1) / kv_keys, pair ? num_sms / 2 : num_sms);
+    return balanced_splits(units, (keys + kv_keys - 1) / kv_keys, pair ? num_sms / 2 : num_sms,
+                           2 * attn::BN / kv_keys);
 }
 
 int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -164,6 +164,9 @@ def test_default_splits_follow_the_kernel_geometry_of_D():
     # take 18 ranges, where 148 single-SM units would take 37
     assert af.splitkv_default_splits(1, 2, 300, 65536, D=128) == 37
     assert af.splitkv_default_splits(1, 2, 300, 65536, D=256) == 18
+    # 64 single-row heads at D = 256: one round of 128 ranges of 128 tiles beats four
+    # of 576 ranges of 29 (a 64-key range's fill is ~4 tiles)
+    assert af.splitkv_default_splits(4, 16, 1, 16384, D=256) == 2
     assert af.ex_default_splits(1, 2, 2, 300, 65536, af.ATTN_MASK_NONE, D=192) == 18
     # head dimensions outside the library's set
     assert af.splitkv_default_splits(1, 4, 1, 16384, D=48) == 0
