@@ -62,8 +62,16 @@ STEP = (("C3", True), ("C4", False), ("C5", True))
 KERNEL_SOURCES = ("attention_forward_18_b200/csrc/attn_fwd_kernel.cuh",
                   "attention_forward_18_b200/csrc/attn_fwd.cu",
                   "attention_forward_18_b200/csrc/ptx.cuh")
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch (ncu, --clock-control none)
-NCU_TRAFFIC = {}
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch (ncu, --clock-control none),
+# with the kernel-source hash of the build captured
+NCU_TRAFFIC = {
+    "C5-causal": {"bytes": 560379648 + 49198336, "src_sha": "3e1f88882f8c27f6",
+                  "note": "ncu --set full, one launch of C5 (read 560.4 MB, write 49.2 MB)"},
+    "C4-noncausal": {"bytes": 402879232 + 111631616, "src_sha": "3e1f88882f8c27f6",
+                     "note": "ncu --set full, one launch of C4 (read 402.9 MB, write 111.6 MB)"},
+    "C3-causal": {"bytes": 539390976 + 47546624, "src_sha": "3e1f88882f8c27f6",
+                  "note": "ncu --set full, one launch of C3 (read 539.4 MB, write 47.5 MB)"},
+}
 
 # North-star fractions of the dense bf16 peak per run (none stated for C1 and C2
 # non-causal).
@@ -338,18 +346,22 @@ def cuda_arm(args, world, rank, local):
 
     peak, peak_kind = tensor_peak()
     per_slot = [sum(t[j] for t in times) / args.steps for j in range(len(launches))]
+    sha = kernel_source_sha()
     per_pass = {}
     for j, (w, c) in enumerate(passes):
         tf = w.flops(c) / (per_slot[j] * 1e-3) / 1e12
+        cap = NCU_TRAFFIC.get(pass_key(w, c))
         per_pass[pass_key(w, c)] = {"ms": round(per_slot[j], 5), "TFLOP/s": round(tf, 1),
-                                    "frac_of_peak": round(tf / peak, 4)}
+                                    "frac_of_peak": round(tf / peak, 4),
+                                    "algorithmic_bytes": w.io_bytes(),
+                                    "traffic": cap["bytes"] if cap and cap["src_sha"] == sha
+                                    else None}
     # dominant kernel: the launch slot with the largest time
     dom = max(range(len(launches)), key=lambda j: per_slot[j])
     dw, dc = passes[dom]
     dom_ms = per_slot[dom]
     achieved = dw.flops(dc) / (dom_ms * 1e-3) / 1e12
     key = pass_key(dw, dc)
-    sha = kernel_source_sha()
     cap = NCU_TRAFFIC.get(key)
     traffic = cap["bytes"] if cap and cap["src_sha"] == sha else None
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
