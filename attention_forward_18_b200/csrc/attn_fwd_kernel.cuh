@@ -357,14 +357,14 @@ __device__ __forceinline__ float softmax_tile_running(uint32_t tS, float c, floa
     uint32_t s[128];
     uint32_t pk[64];
     uint64_t acc = ptx::f32x2(0.f, 0.f);
+    // both halves in one wait: a split load whose second half ran under the first
+    // half's exponentials still waited ~160 clocks for it (measured)
     load_scores<NEG>(tS, s, 0);
+    load_scores<NEG>(tS, s, 1);
     ptx::tmem_wait_ld();
     scores_ready<NEG>(s, 0);
-    // the second half's load runs under the first half's exponentials
-    load_scores<NEG>(tS, s, 1);
-    exp_pairs32<IS_BF16>(s, 0, c, -m_used, pk, acc);
-    ptx::tmem_wait_ld();
     scores_ready<NEG>(s, 1);
+    exp_pairs32<IS_BF16>(s, 0, c, -m_used, pk, acc);
     exp_pairs32<IS_BF16>(s, 32, c, -m_used, pk, acc);
     float alpha = 1.f;
     if (__any_sync(0xffffffffu, sum_pair(acc) > LIMIT)) {
