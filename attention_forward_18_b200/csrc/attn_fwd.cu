@@ -166,6 +166,57 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return x < y + nb && y < x + na;
 }
 
+// Chunks of heads attn_fwd_host pipelines its copies over: at most 8, each at least
+// 8 MB of Q, K and V (below that a copy's fixed cost outweighs the overlap), one for
+// small passes.
+int host_chunks(int BH, int Sq, int Sk, int D) {
+    const int64_t in_bytes = static_cast<int64_t>(BH) * (Sq + 2 * static_cast<int64_t>(Sk)) * D * 2;
+    int64_t n = in_bytes / (8ll << 20);
+    if (n > 8) n = 8;
+    if (n > BH) n = BH;
+    if (n < 1) n = 1;
+    const int per = static_cast<int>((BH + n - 1) / n);
+    return (BH + per - 1) / per;
+}
+
+// attn_fwd_host's two copy streams (non-blocking) and the events that order them
+// against the caller's stream: created once per device on first use and kept for the
+// life of the process (not valid across cudaDeviceReset); `mu` keeps one call's
+// records and waits together.
+struct HostPipe {
+    cudaStream_t in_stream = nullptr, out_stream = nullptr;
+    cudaEvent_t start = nullptr, in = nullptr, out = nullptr, end = nullptr;
+    std::mutex mu;
+};
+
+int host_pipe(HostPipe** out) {
+    static HostPipe pipes[kMaxDevices];
+    static int state[kMaxDevices];  // 0 not made, 1 ready, -1 failed
+    static std::mutex mu;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return ATTN_ERR_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (state[dev] == 0) {
+        HostPipe& p = pipes[dev];
+        const unsigned ef = cudaEventDisableTiming;
+        const bool made =
+            cudaStreamCreateWithFlags(&p.in_stream, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&p.out_stream, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.start, ef) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.in, ef) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.out, ef) == cudaSuccess &&
+            cudaEventCreateWithFlags(&p.end, ef) == cudaSuccess;
+        if (!made) cudaGetLastError();
+        state[dev] = made ? 1 : -1;
+    }
+    if (state[dev] != 1) return ATTN_ERR_LAUNCH;
+    *out = &pipes[dev];
+    return ATTN_OK;
+}
+
 // Hkv: heads of K and V (a divisor of H; H for plain multi-head attention).
 int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
              int B, int H, int Hkv, int Sq, int Sk, int D, float scale, int dtype) {
@@ -578,23 +629,74 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
     if (rc != ATTN_OK) return rc;
     if ((rc = check_device(nullptr)) != ATTN_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t bh = static_cast<size_t>(B) * H;
-    const size_t nq = bh * Sq * D * 2, nk = bh * Sk * D * 2;
-    if (cudaMemcpyAsync(q_dev, q_host, nq, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(k_dev, k_host, nk, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(v_dev, v_host, nk, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_LAUNCH;
+    const int BH = B * H;
+    const bool lse_out = lse_host && lse_dev;
+    const int n = host_chunks(BH, Sq, Sk, D);
+    const int per = (BH + n - 1) / n;
+    // heads [h0, h0 + nh) of the flattened [B*H] axis: contiguous in every tensor
+    auto h2d = [&](int h0, int nh, cudaStream_t st) {
+        const size_t oq = static_cast<size_t>(h0) * Sq * D * 2, ok = static_cast<size_t>(h0) * Sk * D * 2;
+        const size_t nq = static_cast<size_t>(nh) * Sq * D * 2, nk = static_cast<size_t>(nh) * Sk * D * 2;
+        return cudaMemcpyAsync(static_cast<char*>(q_dev) + oq, static_cast<const char*>(q_host) + oq,
+                               nq, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+               cudaMemcpyAsync(static_cast<char*>(k_dev) + ok, static_cast<const char*>(k_host) + ok,
+                               nk, cudaMemcpyHostToDevice, st) == cudaSuccess &&
+               cudaMemcpyAsync(static_cast<char*>(v_dev) + ok, static_cast<const char*>(v_host) + ok,
+                               nk, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    };
+    auto d2h = [&](int h0, int nh, cudaStream_t st) {
+        const size_t oq = static_cast<size_t>(h0) * Sq * D * 2, nq = static_cast<size_t>(nh) * Sq * D * 2;
+        const size_t ol = static_cast<size_t>(h0) * Sq, nl = static_cast<size_t>(nh) * Sq * 4;
+        return cudaMemcpyAsync(static_cast<char*>(o_host) + oq, static_cast<const char*>(o_dev) + oq,
+                               nq, cudaMemcpyDeviceToHost, st) == cudaSuccess &&
+               (!lse_out || cudaMemcpyAsync(lse_host + ol, lse_dev + ol, nl,
+                                            cudaMemcpyDeviceToHost, st) == cudaSuccess);
+    };
+    auto pass = [&](int h0, int nh) {
+        const size_t oq = static_cast<size_t>(h0) * Sq * D * 2, ok = static_cast<size_t>(h0) * Sk * D * 2;
+        return run(static_cast<const char*>(q_dev) + oq, static_cast<const char*>(k_dev) + ok,
+                   static_cast<const char*>(v_dev) + ok, static_cast<char*>(o_dev) + oq,
+                   lse_dev ? lse_dev + static_cast<size_t>(h0) * Sq : nullptr, 1, nh, nh, Sq,
+                   Sk, D, mask_of(causal), scale, dtype, s, 0u);
+    };
+    if (n == 1) {
+        if (!h2d(0, BH, s)) {
+            cudaGetLastError();
+            return ATTN_ERR_LAUNCH;
+        }
+        if ((rc = pass(0, BH)) != ATTN_OK) return rc;
+        if (!d2h(0, BH, s)) {
+            cudaGetLastError();
+            return ATTN_ERR_LAUNCH;
+        }
+        return ATTN_OK;
     }
-    rc = run(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, H, Sq, Sk, D, mask_of(causal), scale,
-             dtype, s, 0u);
+    // Head chunks in a three-stage pipeline: chunk c+1's inputs cross the host link on
+    // one copy stream while chunk c's pass runs on `stream` and chunk c-1's outputs
+    // return on another, so the two directions of the link and the kernel overlap.
+    HostPipe* hp = nullptr;
+    if ((rc = host_pipe(&hp)) != ATTN_OK) return rc;
+    std::lock_guard<std::mutex> lock(hp->mu);
+    bool ok = cudaEventRecord(hp->start, s) == cudaSuccess &&
+              cudaStreamWaitEvent(hp->in_stream, hp->start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(hp->out_stream, hp->start, 0) == cudaSuccess;
+    for (int h0 = 0; ok && h0 < BH; h0 += per) {
+        const int nh = BH - h0 < per ? BH - h0 : per;
+        ok = h2d(h0, nh, hp->in_stream) && cudaEventRecord(hp->in, hp->in_stream) == cudaSuccess &&
+             cudaStreamWaitEvent(s, hp->in, 0) == cudaSuccess;
+        if (ok && (rc = pass(h0, nh)) != ATTN_OK) break;
+        ok = ok && cudaEventRecord(hp->out, s) == cudaSuccess &&
+             cudaStreamWaitEvent(hp->out_stream, hp->out, 0) == cudaSuccess &&
+             d2h(h0, nh, hp->out_stream);
+    }
+    // both copy streams rejoin `stream` on every path, so that the caller's stream
+    // orders everything this call queued (and a capture into a graph stays joined)
+    const bool joined = cudaEventRecord(hp->in, hp->in_stream) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, hp->in, 0) == cudaSuccess &&
+                        cudaEventRecord(hp->end, hp->out_stream) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, hp->end, 0) == cudaSuccess;
     if (rc != ATTN_OK) return rc;
-    if (cudaMemcpyAsync(o_host, o_dev, nq, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
-        cudaGetLastError();
-        return ATTN_ERR_LAUNCH;
-    }
-    if (lse_host && lse_dev &&
-        cudaMemcpyAsync(lse_host, lse_dev, bh * Sq * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    if (!ok || !joined) {
         cudaGetLastError();
         return ATTN_ERR_LAUNCH;
     }

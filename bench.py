@@ -453,8 +453,9 @@ def e2e_arm(af, passes, host, dev, sptr, args, world):
     return {"value": round(world * flops_step * steps / (ms * 1e-3) / 1e12, 4),
             "unit": "TFLOP/s", "steps": steps,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "path": "attn_fwd_host per pass (pinned host buffers, copies + kernel on one "
-                    "stream)" + ("; passes on the same tensors each copy them in"
+            "path": "attn_fwd_host per pass (pinned host buffers; a pass of 16 MB or more "
+                    "of Q, K, V runs as up to 8 head chunks, copies in and out on the "
+                    "library's two copy streams overlapping the kernel)" + ("; passes on the same tensors each copy them in"
                                  if shared else "")}
 
 

@@ -95,10 +95,20 @@ int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
 /*
  * attn_fwd_host -- the same pass from host buffers: copies q, k, v host -> device
  * staging buffers, runs attn_fwd, copies o (and lse when both lse pointers are
- * non-null) back, all queued on `stream`; the caller synchronises the stream before
+ * non-null) back, all ordered on `stream`; the caller synchronises the stream before
  * reading o_host / lse_host.  Host buffers should be page-locked for the copies to
  * be asynchronous.  The staging buffers (q_dev ... lse_dev) are caller-allocated
  * device memory with the shapes and alignment attn_fwd requires.
+ * A pass of at least 16 MB of q, k and v runs as up to 8 chunks of whole heads in a
+ * pipeline: a chunk's inputs are copied in on one of the library's copy streams while
+ * the previous chunk's pass runs on `stream` and the chunk before it is copied out on
+ * the other, so both directions of the host link and the kernel overlap.  The two
+ * copy streams (non-blocking) and four events are created on the current device at
+ * the first such call and kept for the life of the process (not valid across
+ * cudaDeviceReset); every copy is joined back into `stream` before the call returns,
+ * on error paths too, so that `stream` orders all of the call's work and a capture of
+ * `stream` into a graph stays joined.  Concurrent calls on one device queue their
+ * chunks one call after the other.
  */
 int attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                   void *o_host, float *lse_host,

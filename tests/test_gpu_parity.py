@@ -137,6 +137,82 @@ def test_host_buffers_entry_point():
     compare(oh.double().numpy(), lh.double().numpy(), o_ref, l_ref, "host entry")
 
 
+HOST_CHUNKED = [
+    # (B, H, Sq, Sk, D, dtype, causal, with_lse): Q + K + V of 16 MB or more, which
+    # attn_fwd_host pipelines in chunks of whole heads (here 2-8 chunks, the last one
+    # shorter where B*H does not divide)
+    (1, 7, 4096, 4096, 128, "bf16", True, True),      # 2 chunks: 4 + 3 heads
+    (3, 5, 1000, 5000, 64, "f16", False, True),       # 2 chunks: 8 + 7
+    (2, 9, 2048, 2048, 128, "bf16", False, False),    # 3 chunks of 6
+    (1, 11, 300, 9000, 96, "f16", True, True),        # 4 chunks: 3 + 3 + 3 + 2
+    (2, 8, 4096, 4096, 128, "bf16", True, True),      # 6 chunks: 5 x 3 + 1
+]
+
+
+@pytest.mark.parametrize("B,H,Sq,Sk,D,dtype,causal,with_lse", HOST_CHUNKED)
+def test_host_buffers_pipelined_chunks(B, H, Sq, Sk, D, dtype, causal, with_lse):
+    """attn_fwd_host on passes large enough to run as a pipeline of head chunks: O and
+    LSE equal the device entry's bit for bit (a head's arithmetic does not depend on
+    which launch runs it), and oracle rows of the first and last head of every possible
+    chunk boundary match within the tolerances."""
+    q, k, v = make_qkv(B, H, Sq, Sk, D, dtype, 40 + H)
+    scale = 1 / np.sqrt(D)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.full((B, H, Sq), 7.0, dtype=torch.float32).pin_memory()
+    staging = (torch.empty_like(q, device="cuda"), torch.empty_like(k, device="cuda"),
+               torch.empty_like(v, device="cuda"), torch.empty_like(q, device="cuda"),
+               torch.empty((B, H, Sq), dtype=torch.float32, device="cuda"))
+    side = torch.cuda.Stream()
+    af.attention_host(qh, kh, vh, staging, causal=causal, scale=scale, out=oh,
+                      lse=lh if with_lse else None, stream=side)
+    side.synchronize()
+    assert af.attn_fwd_status() == 0
+    o_dev, l_dev = af.attention(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o_dev.cpu())
+    if with_lse:
+        assert torch.equal(lh, l_dev.cpu())
+    else:
+        assert bool((lh == 7.0).all())  # no LSE pointer: the host buffer is untouched
+    heads = sorted({0, B * H - 1} | {x for c in range(1, 9) for x in
+                                     (c * -(-B * H // c) - 1, c * -(-B * H // c))
+                                     if 0 <= x < B * H})
+    rng = np.random.default_rng(B * H)
+    rows = [(bh // H, bh % H, int(i)) for bh in heads
+            for i in {0, Sq - 1, *rng.integers(0, Sq, 3).tolist()}]
+    o_ref, l_ref = oracle.attn_ref_rows(q.double().numpy(), k.double().numpy(),
+                                        v.double().numpy(), np.array(rows), causal, scale)
+    o_got = np.stack([oh[b, h, i].double().numpy() for b, h, i in rows])
+    l_got = np.array([lh[b, h, i].item() for b, h, i in rows]) if with_lse else None
+    compare(o_got, l_got, o_ref, l_ref, "pipelined host entry")
+
+
+def test_host_buffers_back_to_back_calls_on_one_stream():
+    """Two pipelined attn_fwd_host calls queued on one stream without a synchronise in
+    between, the second on other inputs but the same staging and host output buffers:
+    the host output holds the second call's result (the calls are ordered on the
+    stream, copy streams included)."""
+    B, H, S, D = 1, 6, 4096, 128
+    q1, k1, v1 = make_qkv(B, H, S, S, D, "bf16", 71)
+    q2, k2, v2 = make_qkv(B, H, S, S, D, "bf16", 72)
+    pinned1 = [t.pin_memory() for t in (q1, k1, v1)]
+    pinned2 = [t.pin_memory() for t in (q2, k2, v2)]
+    oh = torch.empty_like(q1).pin_memory()
+    lh = torch.empty((B, H, S), dtype=torch.float32).pin_memory()
+    staging = (torch.empty_like(q1, device="cuda"), torch.empty_like(k1, device="cuda"),
+               torch.empty_like(v1, device="cuda"), torch.empty_like(q1, device="cuda"),
+               torch.empty((B, H, S), dtype=torch.float32, device="cuda"))
+    s = torch.cuda.current_stream()
+    af.attention_host(*pinned1, staging, causal=True, out=oh, lse=lh, stream=s)
+    af.attention_host(*pinned2, staging, causal=False, out=oh, lse=lh, stream=s)
+    s.synchronize()
+    o_dev, l_dev = af.attention(q2.cuda(), k2.cuda(), v2.cuda(), causal=False)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o_dev.cpu())
+    assert torch.equal(lh, l_dev.cpu())
+
+
 def test_concurrent_streams_do_not_interfere():
     """The library keeps no per-call state on the device: four passes of different
     shapes, masks and paths (whole, split, grouped heads) in flight at once on four
