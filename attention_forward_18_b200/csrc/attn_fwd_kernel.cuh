@@ -828,15 +828,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int j = 0; ok && j < n; ++j) {
                         const int t = j & 1, i = j >> 1;
                         if (!(ok = wait_bounded(ctx, B_VF(slot(j)), phase(j)))) break;
-                        if (!(ok = wait_bounded(ctx, B_PF(t), pit[t] & 1))) break;
-                        ++pit[t];
+                        // t is a run-time value here: the counters are picked by selects (an
+                        // index by t would put them in local memory, on this thread's path)
+                        if (!(ok = wait_bounded(ctx, B_PF(t), (t ? pit[1] : pit[0]) & 1))) break;
+                        if (t) ++pit[1];
+                        else ++pit[0];
                         // the first P V into O_t overwrites it: the epilogue must have read
                         // the previous unit's O_t
-                        if (i == 0 && !(ok = wait_bounded(ctx, B_OE(t), (ut[t] & 1) ^ 1))) break;
+                        if (i == 0 &&
+                            !(ok = wait_bounded(ctx, B_OE(t), ((t ? ut[1] : ut[0]) & 1) ^ 1)))
+                            break;
                         ptx::tc_fence_after();
                         issue_pv(t, slot(j), i == 0);
                         ptx::mma_commit(B_VE(slot(j)));
-                        if (i == nt[t] - 1) ptx::mma_commit(B_OF(t));
+                        if (i == (t ? nt[1] : nt[0]) - 1) ptx::mma_commit(B_OF(t));
                         if (j + 2 < n) {
                             if (!(ok = wait_bounded(ctx, B_KF(slot(j + 2)), phase(j + 2)))) break;
                             ptx::tc_fence_after();
