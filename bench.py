@@ -65,12 +65,12 @@ KERNEL_SOURCES = ("attention_forward_18_b200/csrc/attn_fwd_kernel.cuh",
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch (ncu, --clock-control none),
 # with the kernel-source hash of the build captured
 NCU_TRAFFIC = {
-    "C5-causal": {"bytes": 560223232 + 50308352, "src_sha": "9091c176c1da1152",
-                  "note": "ncu --set full, one launch of C5 (read 560.2 MB, write 50.3 MB)"},
-    "C4-noncausal": {"bytes": 402737152 + 112028672, "src_sha": "9091c176c1da1152",
-                     "note": "ncu --set full, one launch of C4 (read 402.7 MB, write 112.0 MB)"},
-    "C3-causal": {"bytes": 529649152 + 47200000, "src_sha": "9091c176c1da1152",
-                  "note": "ncu --set full, one launch of C3 (read 529.6 MB, write 47.2 MB)"},
+    "C5-causal": {"bytes": 567774720 + 49346816, "src_sha": "c7d778ee895f2184",
+                  "note": "ncu --set full, one launch of C5 (read 567.8 MB, write 49.3 MB)"},
+    "C4-noncausal": {"bytes": 402735872 + 111735040, "src_sha": "c7d778ee895f2184",
+                     "note": "ncu --set full, one launch of C4 (read 402.7 MB, write 111.7 MB)"},
+    "C3-causal": {"bytes": 525650944 + 47049728, "src_sha": "c7d778ee895f2184",
+                  "note": "ncu --set full, one launch of C3 (read 525.7 MB, write 47.0 MB)"},
 }
 
 # North-star fractions of the dense bf16 peak per run (none stated for C1 and C2
