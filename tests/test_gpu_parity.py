@@ -213,6 +213,77 @@ def test_host_buffers_back_to_back_calls_on_one_stream():
     assert torch.equal(lh, l_dev.cpu())
 
 
+def _host_case(B, H, S, D, seed):
+    q, k, v = make_qkv(B, H, S, S, D, "bf16", seed)
+    pinned = [t.pin_memory() for t in (q, k, v)]
+    oh = torch.zeros_like(q).pin_memory()
+    lh = torch.zeros((B, H, S), dtype=torch.float32).pin_memory()
+    staging = (torch.empty_like(q, device="cuda"), torch.empty_like(k, device="cuda"),
+               torch.empty_like(v, device="cuda"), torch.empty_like(q, device="cuda"),
+               torch.empty((B, H, S), dtype=torch.float32, device="cuda"))
+    return (q, k, v), pinned, oh, lh, staging
+
+
+def test_host_buffers_pipeline_in_a_cuda_graph():
+    """A pipelined attn_fwd_host call captured into a CUDA graph (its copy streams join
+    the capture and rejoin the captured stream), replayed on new host inputs written
+    into the same pinned buffers: each replay's host output equals the device entry's."""
+    B, H, S, D = 1, 6, 4096, 128
+    (q, k, v), pinned, oh, lh, staging = _host_case(B, H, S, D, 81)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        af.attention_host(*pinned, staging, causal=True, out=oh, lse=lh, stream=side)  # warm-up
+    side.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        af.attention_host(*pinned, staging, causal=True, out=oh, lse=lh,
+                          stream=torch.cuda.current_stream())
+    for seed in (82, 83):
+        q2, k2, v2 = make_qkv(B, H, S, S, D, "bf16", seed)
+        for dst, src in zip(pinned, (q2, k2, v2)):
+            dst.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert af.attn_fwd_status() == 0
+        o_dev, l_dev = af.attention(q2.cuda(), k2.cuda(), v2.cuda(), causal=True)
+        torch.cuda.synchronize()
+        assert torch.equal(oh, o_dev.cpu()) and torch.equal(lh, l_dev.cpu())
+    del graph
+
+
+def test_host_buffers_pipeline_from_two_threads():
+    """Two host threads calling the pipelined attn_fwd_host at once, each on its own
+    stream and buffers (the calls on one device queue one after the other): both host
+    outputs equal the device entry's."""
+    import threading
+    cases = [_host_case(1, 6, 4096, 128, 91), _host_case(2, 3, 4096, 128, 92)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    errors = []
+
+    def worker(i):
+        try:
+            _, pinned, oh, lh, staging = cases[i]
+            for _ in range(3):
+                af.attention_host(*pinned, staging, causal=bool(i), out=oh, lse=lh,
+                                  stream=streams[i])
+            streams[i].synchronize()
+        except Exception as e:  # reported in the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    assert af.attn_fwd_status() == 0
+    for i, ((q, k, v), _, oh, lh, _) in enumerate(cases):
+        o_dev, l_dev = af.attention(q.cuda(), k.cuda(), v.cuda(), causal=bool(i))
+        torch.cuda.synchronize()
+        assert torch.equal(oh, o_dev.cpu()) and torch.equal(lh, l_dev.cpu())
+
+
 def test_concurrent_streams_do_not_interfere():
     """The library keeps no per-call state on the device: four passes of different
     shapes, masks and paths (whole, split, grouped heads) in flight at once on four
